@@ -1,0 +1,132 @@
+"""ctypes binding of ``libfp8adam.so`` (C ABI in include/fp8adam.h).
+
+Argument marshalling only: every function forwards to the C entry point of
+the same name, and every step of the optimizer runs in the library's CUDA
+kernels.  There is no fallback: if the library is missing, loading raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfp8adam.so")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED_FMT = -2
+ERR_CUDA = -3
+ERR_OOM = -4
+ERR_WRONG_DEVICE = -5
+
+E4M3, E5M2, FP32 = 0, 1, 2
+FLAG_STATS = 1
+FLAG_JIT_EVERY_STEP = 2
+
+
+class fp8adam_tensor(ctypes.Structure):
+    _fields_ = [("param", ctypes.c_void_p), ("grad", ctypes.c_void_p), ("m", ctypes.c_void_p),
+                ("v", ctypes.c_void_p), ("numel", ctypes.c_int64)]
+
+
+class Fp8AdamError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__("%s failed: %s (%d)" % (fn, fp8adam_strerror(code), code))
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libfp8adam.so is not built (python -m fp8_quantized_adam_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, u32, f = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float
+        L.fp8adam_create.restype = ctypes.c_int
+        L.fp8adam_create.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, vp, vp, vp, vp, i32, i32, u32,
+                                     ctypes.POINTER(vp)]
+        L.fp8adam_step.restype = ctypes.c_int
+        L.fp8adam_step.argtypes = [vp, f, f, f, f, f, i64, vp]
+        L.fp8adam_get_stats.restype = ctypes.c_int
+        L.fp8adam_get_stats.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), vp]
+        L.fp8adam_reset_stats.restype = ctypes.c_int
+        L.fp8adam_reset_stats.argtypes = [vp, vp]
+        L.fp8adam_destroy.restype = ctypes.c_int
+        L.fp8adam_destroy.argtypes = [vp]
+        L.fp8adam_strerror.restype = ctypes.c_char_p
+        L.fp8adam_strerror.argtypes = [ctypes.c_int]
+        L.fp8adam_encode.restype = ctypes.c_int
+        L.fp8adam_encode.argtypes = [i32, vp, vp, i64, i32, vp]
+        L.fp8adam_encode_bits_range.restype = ctypes.c_int
+        L.fp8adam_encode_bits_range.argtypes = [i32, u32, i64, vp, i32, vp]
+        L.fp8adam_decode.restype = ctypes.c_int
+        L.fp8adam_decode.argtypes = [i32, vp, vp, i64, i32, vp]
+        L.fp8adam_launch_count.restype = ctypes.c_uint64
+        L.fp8adam_launch_count.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, rc: int) -> int:
+    if rc != OK:
+        raise Fp8AdamError(fn, rc)
+    return rc
+
+
+# ---- the C entry points, same names --------------------------------------
+def fp8adam_strerror(code: int) -> str:
+    return lib().fp8adam_strerror(code).decode()
+
+
+def fp8adam_create(tensors, num_tensors: int, scale_m: int, scale_v: int, amax_m: int, amax_v: int,
+                   m_fmt: int, v_fmt: int, flags: int) -> int:
+    """tensors: a ctypes array of fp8adam_tensor; pointers are ints.
+    Returns the context handle (int)."""
+    out = ctypes.c_void_p()
+    _check("fp8adam_create", lib().fp8adam_create(tensors, num_tensors, scale_m, scale_v, amax_m, amax_v,
+                                                  m_fmt, v_fmt, flags, ctypes.byref(out)))
+    return out.value
+
+
+def fp8adam_step(ctx: int, lr: float, beta1: float, beta2: float, eps: float, weight_decay: float,
+                 step: int, cuda_stream: int) -> None:
+    _check("fp8adam_step", lib().fp8adam_step(ctx, lr, beta1, beta2, eps, weight_decay, step, cuda_stream))
+
+
+def fp8adam_get_stats(ctx: int, cuda_stream: int):
+    out = (ctypes.c_uint64 * 2)()
+    _check("fp8adam_get_stats", lib().fp8adam_get_stats(ctx, out, cuda_stream))
+    return int(out[0]), int(out[1])
+
+
+def fp8adam_reset_stats(ctx: int, cuda_stream: int) -> None:
+    _check("fp8adam_reset_stats", lib().fp8adam_reset_stats(ctx, cuda_stream))
+
+
+def fp8adam_destroy(ctx: int) -> None:
+    _check("fp8adam_destroy", lib().fp8adam_destroy(ctx))
+
+
+def fp8adam_encode(fmt: int, x: int, out: int, n: int, impl: int, cuda_stream: int) -> None:
+    _check("fp8adam_encode", lib().fp8adam_encode(fmt, x, out, n, impl, cuda_stream))
+
+
+def fp8adam_encode_bits_range(fmt: int, first: int, n: int, out: int, impl: int, cuda_stream: int) -> None:
+    _check("fp8adam_encode_bits_range", lib().fp8adam_encode_bits_range(fmt, first, n, out, impl, cuda_stream))
+
+
+def fp8adam_decode(fmt: int, codes: int, out: int, n: int, impl: int, cuda_stream: int) -> None:
+    _check("fp8adam_decode", lib().fp8adam_decode(fmt, codes, out, n, impl, cuda_stream))
+
+
+def fp8adam_launch_count() -> int:
+    return int(lib().fp8adam_launch_count())
+
+
+EXPORTED = ["fp8adam_create", "fp8adam_step", "fp8adam_get_stats", "fp8adam_reset_stats",
+            "fp8adam_destroy", "fp8adam_strerror", "fp8adam_encode", "fp8adam_encode_bits_range",
+            "fp8adam_decode", "fp8adam_launch_count"]

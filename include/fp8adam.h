@@ -1,0 +1,158 @@
+/*
+ * fp8adam.h -- C ABI of the B200 (sm_100a) AdamW step with FP8-stored
+ * moments.
+ *
+ * What the library computes (sources cited by page title and section):
+ *   - "Scaling FP8 training to trillion-token LLMs" (abstract): both Adam
+ *     moments are quantised to FP8.
+ *   - blog.daoxuan.cc explainer of that paper, section "Adam 为什么给第一矩选
+ *     E4M3、第二矩选 E5M2": the first moment m is stored in E4M3 (precision),
+ *     the second moment v in E5M2 (range); sub-section "两种 FP8 格式差在指数位
+ *     和尾数位" gives the two bit layouts.
+ *   - "FP8训练的稳定性挑战：E5M2与E4M3格式在梯度更新与前向传播中的混合精度策略",
+ *     section "代码示例" (optim.AdamW) for the update, section
+ *     "应对FP8训练稳定性挑战的策略" (amax-tracked range and exponent-bias
+ *     adjustment) and its transformer_engine example (DelayedScaling,
+ *     margin 0) for the per-tensor scale.
+ *
+ * One step, per tensor i and element j (all fp32, no FMA contraction):
+ *   g      = bf16 gradient widened to fp32
+ *   m_old  = dec(qm) / scale_m[i]          v_old = dec(qv) / scale_v[i]
+ *   m      = b1*m_old + (1-b1)*g            v     = b2*v_old + (1-b2)*g*g
+ *   amax_m[i] = max|m|, amax_v[i] = max|v| over the tensor (unquantised)
+ *   s'     = largest 2^k, |k| <= 126, with amax_prev * 2^k <= max of the
+ *            format (448 for E4M3, 57344 for E5M2); amax_prev is the previous
+ *            step's amax, or this step's own at step 1 (a pre-pass); an amax
+ *            of 0, inf or NaN keeps the previous scale
+ *   qm     = enc(m * s'_m)                  qv    = enc(v * s'_v)
+ *            (round to nearest, ties to even code, saturate to +-max, NaN
+ *            -> NaN code)
+ *   p      = p*(1 - lr*wd) - (lr/(1-b1^t)) * m / (sqrt(v)/sqrt(1-b2^t) + eps)
+ *            evaluated as den = sqrtf(v)*isbc2; den = den + eps; u = m/den;
+ *            p = p*decay; p = p - step_size*u, with isbc2, step_size and
+ *            decay computed in double on the host and rounded once to fp32.
+ *   scale_m[i] = s'_m, scale_v[i] = s'_v after the step.
+ * The update uses this step's unquantised m and v; the FP8 codes carry them
+ * to the next step.
+ *
+ * Memory and ownership.  The caller owns every tensor buffer: params (fp32),
+ * grads (bf16 bit patterns), m and v (uint8 codes, or fp32 in FP8ADAM_FP32
+ * mode), and the per-tensor arrays scale_m/scale_v/amax_m/amax_v (fp32,
+ * num_tensors each).  All are device pointers, fixed from create to destroy.
+ * Initial state: codes 0, scales 1.0, amax 0.0.  The context owns its
+ * device-side tables and accumulators.
+ *
+ * Threading.  A context is used from one host thread and one stream at a
+ * time.  fp8adam_step is asynchronous on the given stream and never
+ * synchronises the host.  The CUDA device current at create must be current
+ * at every call.
+ *
+ * Errors.  Every function returns FP8ADAM_OK (0) or a negative code; argument
+ * errors are detected on the host before any GPU work is queued.
+ */
+#ifndef FP8ADAM_H
+#define FP8ADAM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP8ADAM_OK 0
+#define FP8ADAM_ERR_INVALID_ARG (-1)     /* null pointer, bad size or hyper-parameter */
+#define FP8ADAM_ERR_UNSUPPORTED_FMT (-2) /* format id not in fp8adam_fmt */
+#define FP8ADAM_ERR_CUDA (-3)            /* a CUDA runtime call failed */
+#define FP8ADAM_ERR_OOM (-4)             /* device allocation failed in create */
+#define FP8ADAM_ERR_WRONG_DEVICE (-5)    /* current device differs from create's */
+
+/* Storage format of a moment. */
+typedef enum {
+  FP8ADAM_E4M3 = 0, /* OCP E4M3 ("fn"): bias 7, max 448, S.1111.111 = NaN, no inf */
+  FP8ADAM_E5M2 = 1, /* E5M2: bias 15, max 57344, IEEE-style inf/NaN */
+  FP8ADAM_FP32 = 2  /* unquantised fp32 moment (reference mode, 4 B/element) */
+} fp8adam_fmt;
+
+/* Flags of fp8adam_create. */
+#define FP8ADAM_FLAG_STATS 1u            /* count flushed v and saturated codes */
+#define FP8ADAM_FLAG_JIT_EVERY_STEP 2u   /* "current" scaling: pre-pass every step */
+
+/* One tensor.  param: fp32[numel]; grad: bf16[numel] (raw bits); m, v:
+ * uint8[numel] codes or fp32[numel] in FP8ADAM_FP32 mode.  Any numel >= 0
+ * (an empty tensor is skipped and its state left as is).  Buffers that are
+ * 16-byte aligned take the vectorised path; others are processed element by
+ * element, with the same results. */
+typedef struct {
+  float* param;
+  const uint16_t* grad;
+  void* m;
+  void* v;
+  int64_t numel;
+} fp8adam_tensor;
+
+typedef struct fp8adam_ctx fp8adam_ctx; /* opaque */
+
+/* Builds the device tensor table and chunk table of a whole parameter list
+ * (one step = one kernel launch over all tensors).  Copies `tensors`
+ * (host array) to the device, allocates the context's accumulators and
+ * synchronises once.  scale_m/scale_v/amax_m/amax_v: device fp32
+ * [num_tensors].  m_fmt/v_fmt: fp8adam_fmt.  Returns INVALID_ARG for null
+ * pointers, num_tensors < 1 or numel < 0; UNSUPPORTED_FMT; OOM; CUDA. */
+int fp8adam_create(const fp8adam_tensor* tensors, int32_t num_tensors,
+                   float* scale_m, float* scale_v, float* amax_m,
+                   float* amax_v, int32_t m_fmt, int32_t v_fmt,
+                   uint32_t flags, fp8adam_ctx** out);
+
+/* One AdamW step (t = step, 1-based) on every tensor of the context, queued
+ * on `cuda_stream` (a cudaStream_t; NULL = legacy default stream).  Requires
+ * 0 <= beta1, beta2 < 1, eps >= 0, finite lr and weight_decay, step >= 1;
+ * otherwise INVALID_ARG with nothing queued.  At step 1 (or every step with
+ * FP8ADAM_FLAG_JIT_EVERY_STEP) an amax pre-pass runs first.  Returns CUDA if
+ * a launch fails. */
+int fp8adam_step(fp8adam_ctx* ctx, float lr, float beta1, float beta2,
+                 float eps, float weight_decay, int64_t step,
+                 void* cuda_stream);
+
+/* Reads the counters accumulated since create or the last reset (only with
+ * FP8ADAM_FLAG_STATS; zeros otherwise): out[0] = v elements with v > 0 whose
+ * code is +-0 ("flushed"), out[1] = elements whose scaled m or v exceeded the
+ * format's max (saturated; one count per moment).  `out` is host memory;
+ * waits for `cuda_stream`. */
+int fp8adam_get_stats(fp8adam_ctx* ctx, uint64_t* out, void* cuda_stream);
+
+/* Zeroes the counters (queued on cuda_stream). */
+int fp8adam_reset_stats(fp8adam_ctx* ctx, void* cuda_stream);
+
+/* Frees the context (synchronises the device first).  NULL is accepted. */
+int fp8adam_destroy(fp8adam_ctx* ctx);
+
+/* Static description of an error code. */
+const char* fp8adam_strerror(int code);
+
+/* ---- device codec (verification entry points) -------------------------
+ * impl 0 = hardware conversion (cvt.rn.satfinite.{e4m3x2,e5m2x2}.f32 /
+ * cvt.rn.f16x2.{e4m3x2,e5m2x2}), impl 1 = integer/bit-manipulation path.
+ * Both implement the codec described above. */
+
+/* out[j] = enc(fmt, x[j]) for j < n; x, out device pointers. */
+int fp8adam_encode(int32_t fmt, const float* x, uint8_t* out, int64_t n,
+                   int32_t impl, void* cuda_stream);
+
+/* out[j] = enc(fmt, float with bit pattern first + j), j < n <= 2^32 - first:
+ * encodes a range of the fp32 bit-pattern space without an input buffer. */
+int fp8adam_encode_bits_range(int32_t fmt, uint32_t first, int64_t n,
+                              uint8_t* out, int32_t impl, void* cuda_stream);
+
+/* out[j] = dec(fmt, codes[j]) as fp32. */
+int fp8adam_decode(int32_t fmt, const uint8_t* codes, float* out, int64_t n,
+                   int32_t impl, void* cuda_stream);
+
+/* Number of kernels launched by the library on this process since load (for
+ * accounting launches inside a timed region). */
+uint64_t fp8adam_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8ADAM_H */

@@ -68,8 +68,8 @@ def rint_encode(fmt: int, x: np.ndarray) -> np.ndarray:
     x = np.asarray(x, np.float32)
     a = np.abs(x).astype(np.float64)
     with np.errstate(invalid="ignore", over="ignore"):
-        _, e = np.frexp(a)
-        eb = np.maximum(e - 1, emin)                   # binade exponent (>= emin)
+        _, e = np.frexp(a)                             # frexp(0) gives e = 0
+        eb = np.maximum(np.where(a > 0, e - 1, emin), emin)  # binade exponent (>= emin)
         n = np.rint(np.ldexp(a, M - eb))               # quanta of 2^(eb-M), exact scaling
         n = np.where(np.isfinite(n), n, 0.0)
         code = ((eb - emin).astype(np.int64) << M) + n.astype(np.int64)

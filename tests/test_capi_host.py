@@ -1,0 +1,82 @@
+"""The C-ABI library on the host (no GPU needed): it loads, exports every
+symbol include/fp8adam.h declares, and rejects bad arguments with error
+codes before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp8_quantized_adam_b200 import build as b
+from fp8_quantized_adam_b200 import capi
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fp8adam.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    b.build()
+    return capi.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8adam_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(capi.EXPORTED) == names
+
+
+def test_strerror(L):
+    assert capi.fp8adam_strerror(0) == "ok"
+    for code in (-1, -2, -3, -4, -5):
+        assert capi.fp8adam_strerror(code) not in ("ok", "unknown error")
+    assert capi.fp8adam_strerror(-99) == "unknown error"
+
+
+def test_create_rejects_bad_arguments_on_host(L):
+    T = capi.fp8adam_tensor * 1
+    out = ctypes.c_void_p()
+    t = T(capi.fp8adam_tensor(8, 8, 8, 8, 16))
+    # null output / tensors / arrays
+    assert L.fp8adam_create(t, 1, 8, 8, 8, 8, 0, 1, 0, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_create(None, 1, 8, 8, 8, 8, 0, 1, 0, ctypes.byref(out)) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_create(t, 1, None, 8, 8, 8, 0, 1, 0, ctypes.byref(out)) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_create(t, 0, 8, 8, 8, 8, 0, 1, 0, ctypes.byref(out)) == capi.ERR_INVALID_ARG
+    # formats and flags
+    assert L.fp8adam_create(t, 1, 8, 8, 8, 8, 3, 1, 0, ctypes.byref(out)) == capi.ERR_UNSUPPORTED_FMT
+    assert L.fp8adam_create(t, 1, 8, 8, 8, 8, 0, -1, 0, ctypes.byref(out)) == capi.ERR_UNSUPPORTED_FMT
+    assert L.fp8adam_create(t, 1, 8, 8, 8, 8, 0, 1, 64, ctypes.byref(out)) == capi.ERR_INVALID_ARG
+    # negative size, null buffer with elements
+    bad = T(capi.fp8adam_tensor(8, 8, 8, 8, -1))
+    assert L.fp8adam_create(bad, 1, 8, 8, 8, 8, 0, 1, 0, ctypes.byref(out)) == capi.ERR_INVALID_ARG
+    bad = T(capi.fp8adam_tensor(8, None, 8, 8, 5))
+    assert L.fp8adam_create(bad, 1, 8, 8, 8, 8, 0, 1, 0, ctypes.byref(out)) == capi.ERR_INVALID_ARG
+    assert out.value is None
+
+
+def test_step_and_codec_reject_bad_arguments_on_host(L):
+    assert L.fp8adam_step(None, 1e-3, 0.9, 0.95, 1e-8, 0.1, 1, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_get_stats(None, None, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_reset_stats(None, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_destroy(None) == capi.OK
+    assert L.fp8adam_encode(2, 8, 8, 4, 0, None) == capi.ERR_UNSUPPORTED_FMT
+    assert L.fp8adam_encode(0, 8, 8, 4, 2, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_encode(0, 8, 8, -1, 0, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_encode(0, 8, 8, 0, 0, None) == capi.OK  # nothing to do
+    assert L.fp8adam_decode(5, 8, 8, 4, 0, None) == capi.ERR_UNSUPPORTED_FMT
+    assert L.fp8adam_encode_bits_range(0, 0xFFFFFFFF, 2, 16, 0, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_encode_bits_range(0, 0, 4, 2, 0, None) == capi.ERR_INVALID_ARG  # misaligned out
+    assert isinstance(capi.fp8adam_launch_count(), int)
+
+
+def test_binding_raises_on_error_codes(L):
+    with pytest.raises(capi.Fp8AdamError) as e:
+        capi.fp8adam_step(0, 1e-3, 0.9, 0.95, 1e-8, 0.1, 1, 0)
+    assert e.value.code == capi.ERR_INVALID_ARG

@@ -1,0 +1,246 @@
+"""The CUDA step against the oracle, element by element, free-running from
+the same seeded state on the same seeded gradients (all calls go through the
+C ABI)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import pins
+from fp8_quantized_adam_b200 import FP8AdamW, capi, workloads
+from gpu_harness import HP, Run, bf16_host_bits
+
+pytestmark = pytest.mark.gpu
+
+E4, E5, F32 = oracle.E4M3, oracle.E5M2, oracle.FP32
+
+
+def test_single_tensor_1m_all_elements_10_steps():
+    """1,048,576 params, g = 10^U(-6,-1) * N(0,1): every element, 10 steps."""
+    r = Run(workloads.layout("single_1m"), workloads.CFG_ID["single_1m"])
+    for _ in range(10):
+        r.step()
+        res = r.compare()
+    assert res["flips"] == 0
+
+
+def test_llama2_100m_layout_subset_100_steps():
+    specs = workloads.layout("llama2_100m")
+    names = [s.name for s in specs]
+    subset = [i for i, s in enumerate(specs) if s.kind == "norm"] + [names.index("l0.q"), names.index("l5.w1")]
+    r = Run(specs, workloads.CFG_ID["llama2_100m"], subset=subset)
+    for t in range(1, 101):
+        r.step()
+        if t in (1, 2, 3, 10, 50, 100):
+            r.compare()
+            r.check_invariants()
+
+
+@pytest.mark.parametrize("fmts", [(E4, E4), (E4, E5), (E5, E4), (E5, E5), (F32, F32)],
+                         ids=["m4v4", "m4v5", "m5v4", "m5v5", "fp32"])
+def test_format_ablation_modes(fmts):
+    specs = workloads.layout("ablation_100m")
+    names = [s.name for s in specs]
+    subset = [names.index("final_norm"), names.index("l3.k"), names.index("l11.w3")]
+    r = Run(specs, workloads.CFG_ID["ablation_100m"], m_fmt=fmts[0], v_fmt=fmts[1], subset=subset)
+    for t in range(1, 21):
+        r.step()
+        if t in (1, 2, 20):
+            r.compare()
+    r.check_invariants()
+
+
+def test_stats_counters_match_oracle():
+    """Flushed-v and saturation counters over a whole model equal the sums of
+    the oracle's per-tensor counters; v in E4M3 flushes more than E5M2."""
+    specs = workloads.custom_layout([70001, 4096, 33, 200000])
+    flushed = {}
+    for vf in (E4, E5):
+        r = Run(specs, 9, m_fmt=E4, v_fmt=vf, stats=True)
+        for t in range(1, 6):
+            r.step()
+        r.compare()
+        got = r.opt.stats()
+        exp = tuple(int(sum(int(r.ref[i].stats[k]) for i in r.subset)) for k in (0, 1))
+        assert got == exp
+        flushed[vf] = got[0]
+    assert flushed[E4] > flushed[E5]
+
+
+def test_current_scaling_every_step():
+    specs = workloads.custom_layout([65536 * 3 + 5, 1000])
+    r = Run(specs, 11, jit_every_step=True)
+    for _ in range(6):
+        r.step()
+        r.compare()
+
+
+def test_edge_sizes_and_misaligned_views():
+    """Sizes around the 16-element vector, the 4096-element CTA tile and the
+    65536-element chunk, an empty tensor, and tensors whose buffers are
+    offset by one element (element-by-element path)."""
+    sizes = [0, 1, 15, 16, 17, 4095, 4096, 4097, 65535, 65536, 65537, 3 * 65536 + 4099]
+    specs = workloads.custom_layout(sizes)
+    r = Run(specs, 12)
+    for _ in range(4):
+        r.step()
+        r.compare()
+    # misaligned: views starting one element into each buffer
+    dev = torch.device("cuda:0")
+    ns = [33, 4097, 70000]
+    p = [torch.zeros(n + 1, device=dev)[1:] for n in ns]
+    g = [torch.zeros(n + 1, device=dev, dtype=torch.bfloat16)[1:] for n in ns]
+    m = [torch.zeros(n + 1, device=dev, dtype=torch.uint8)[1:] for n in ns]
+    v = [torch.zeros(n + 1, device=dev, dtype=torch.uint8)[1:] for n in ns]
+    specs2 = workloads.custom_layout(ns)
+    workloads.init_params_into(specs2, p, 13)
+    opt = FP8AdamW(p, g, m=m, v=v)
+    ref = [oracle.TensorState(x.cpu().numpy(), E4, E5) for x in p]
+    sig = workloads.tensor_sigmas(specs2, 13)
+    for t in range(1, 4):
+        workloads.grads_into(specs2, g, 13, t, sig)
+        opt.step()
+        for i, rs in enumerate(ref):
+            rs.step(bf16_host_bits(g[i]), HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], t)
+    torch.cuda.synchronize()
+    for i, rs in enumerate(ref):
+        assert (m[i].cpu().numpy() == rs.m).all() and (v[i].cpu().numpy() == rs.v).all()
+        assert (p[i].cpu().numpy().view(np.uint32) == rs.p.view(np.uint32)).all()
+        assert float(opt.amax_m[i]) == float(rs.amax_m[0]) and float(opt.scale_v[i]) == float(rs.scale_v[0])
+
+
+def test_zero_gradients_keep_scale_and_decay_params():
+    specs = workloads.custom_layout([5000])
+    r = Run(specs, 14)
+    for t in range(1, 4):
+        r.t += 1
+        r.model.g.zero_()
+        r.opt.step()
+        r.oracle_step()
+        r.compare()
+    assert float(r.model.scale_m[0]) == 1.0 and float(r.model.amax_m[0]) == 0.0
+
+
+def test_nan_gradient_reaches_amax_without_fault():
+    specs = workloads.custom_layout([10000, 300])
+    r = Run(specs, 15)
+    r.step()
+    r.t += 1
+    r.draw_grads(r.t)
+    r.model.g[1234] = float("nan")
+    r.opt.step()
+    r.oracle_step()
+    r.compare()
+    assert math.isnan(float(r.model.amax_m[0])) and math.isfinite(float(r.model.amax_m[1]))
+    r.step()  # a NaN amax keeps the previous scale; the NaN element stays NaN
+    r.compare()
+
+
+def test_checkpoint_resume_is_bitwise():
+    specs = workloads.custom_layout([100000, 4096, 77])
+    a = Run(specs, 16, subset=[])
+    for _ in range(10):
+        a.step(with_oracle=False)
+    b = Run(specs, 16, subset=[])
+    for _ in range(5):
+        b.step(with_oracle=False)
+    sd = b.opt.state_dict()
+    c = Run(specs, 16, subset=[])  # a fresh optimizer on fresh buffers, then restore
+    c.opt.load_state_dict(sd)
+    c.t = b.t
+    for _ in range(5):
+        c.step(with_oracle=False)
+    torch.cuda.synchronize()
+    for x, y in ((a.model.p, c.model.p), (a.model.m, c.model.m), (a.model.v, c.model.v),
+                 (a.model.scale_m, c.model.scale_m), (a.model.amax_v, c.model.amax_v)):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+
+
+def test_two_runs_are_bitwise_identical():
+    specs = workloads.layout("single_1m")
+    runs = []
+    for _ in range(2):
+        r = Run(specs, 1, subset=[])
+        for _ in range(5):
+            r.step(with_oracle=False)
+        torch.cuda.synchronize()
+        runs.append(r)
+    for name in ("p", "m", "v", "scale_m", "scale_v", "amax_m", "amax_v"):
+        assert torch.equal(getattr(runs[0].model, name).view(torch.uint8),
+                           getattr(runs[1].model, name).view(torch.uint8)), name
+
+
+def test_step_argument_errors_queue_nothing():
+    specs = workloads.custom_layout([64])
+    r = Run(specs, 17, subset=[])
+    before = capi.fp8adam_launch_count()
+    for kw in (dict(step=0), dict(beta1=1.0), dict(beta2=-0.1), dict(eps=-1.0), dict(lr=float("nan"))):
+        args = dict(lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.0, step=1)
+        args.update(kw)
+        with pytest.raises(capi.Fp8AdamError) as e:
+            capi.fp8adam_step(r.opt.ctx, args["lr"], args["beta1"], args["beta2"], args["eps"],
+                              args["weight_decay"], args["step"], 0)
+        assert e.value.code == capi.ERR_INVALID_ARG
+    assert capi.fp8adam_launch_count() == before
+
+
+@pytest.mark.slow
+def test_int64_indexing_beyond_2_pow_31():
+    """A 2^31 + 3*4096 + 5 element tensor with inputs periodic in 4096
+    elements: outputs are periodic too, so elements past index 2^31 must
+    equal the oracle run on one period (same amax, same per-element math)."""
+    period = 4096
+    n = (1 << 31) + 3 * period + 5
+    dev = torch.device("cuda:0")
+    base_specs = workloads.custom_layout([period])
+    pp = torch.zeros(period)
+    workloads.init_params_into(base_specs, [pp], 18)
+    sig = workloads.tensor_sigmas(base_specs, 18)
+    gg = [torch.zeros(period, dtype=torch.bfloat16) for _ in range(2)]
+    for t in (1, 2):
+        workloads.grads_into(base_specs, [gg[t - 1]], 18, t, sig)
+    reps = (n + period - 1) // period
+    p = pp.to(dev).repeat(reps)[:n].contiguous()
+    g = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    m = torch.zeros(n, dtype=torch.uint8, device=dev)
+    v = torch.zeros(n, dtype=torch.uint8, device=dev)
+    opt = FP8AdamW([p], [g], m=[m], v=[v])
+    ref = oracle.TensorState(pp.numpy(), E4, E5)
+    for t in (1, 2):
+        g.copy_(gg[t - 1].to(dev).repeat(reps)[:n])
+        opt.step()
+        ref.step(bf16_host_bits(gg[t - 1]), HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], t)
+    torch.cuda.synchronize()
+    for start in ((1 << 31) - period, (1 << 31), n - 5 - period):
+        k = start - start % period
+        assert (m[k:k + period].cpu().numpy() == ref.m).all()
+        assert (v[k:k + period].cpu().numpy() == ref.v).all()
+        assert (p[k:k + period].cpu().numpy().view(np.uint32) == ref.p.view(np.uint32)).all()
+    tail = n - (n // period) * period
+    assert (m[n - tail:].cpu().numpy() == ref.m[:tail]).all()
+    assert float(opt.amax_m[0]) == float(ref.amax_m[0]) and float(opt.scale_v[0]) == float(ref.scale_v[0])
+
+
+@pytest.mark.slow
+def test_stress_20k_tensors_full_parity_2_steps():
+    """20,000 x 4096 + 8 x 2^28 in one launch per step; every element of
+    every tensor against the oracle (run on all host cores)."""
+    r = Run(workloads.layout("stress_20k"), workloads.CFG_ID["stress_20k"])
+    for _ in range(2):
+        r.step()
+        res = r.compare()
+    assert res["elements"] == workloads.total_params(r.specs)
+
+
+@pytest.mark.slow
+def test_llama2_7b_layout_subset_3_steps():
+    specs = workloads.layout("llama2_7b")
+    names = [s.name for s in specs]
+    subset = [i for i, s in enumerate(specs) if s.kind == "norm"] + [names.index("l0.q"), names.index("l31.w2")]
+    r = Run(specs, workloads.CFG_ID["llama2_7b"], subset=subset)
+    for _ in range(3):
+        r.step()
+        r.compare()
+        r.check_invariants()
