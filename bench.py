@@ -172,7 +172,9 @@ def run_oracle_sample(name: str, steps: int, warmup: int):
 
 
 def reference_arm(args):
-    rank = int(os.environ.get("RANK", "0"))
+    from fp8_quantized_adam_b200 import ranks
+
+    _, rank, _ = ranks.env()
     if rank != 0:
         return
     import oracle
@@ -204,23 +206,17 @@ def workload_config(name: str, n: int) -> dict:
 # ----------------------------------------------------------------- our arm
 def our_arm(args):
     import torch
-    import torch.distributed as dist
 
-    from fp8_quantized_adam_b200 import FP8AdamW, build, capi, workloads
+    from fp8_quantized_adam_b200 import FP8AdamW, build, capi, ranks, workloads
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = ranks.env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    ranks.init("nccl", dev)
     build.build()
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        ranks.barrier()
         torch.cuda.synchronize()
 
     name = args.workload
@@ -228,9 +224,10 @@ def our_arm(args):
     cfg = workloads.CFG_ID[name]
     n_params = workloads.total_params(specs)
     model = workloads.FlatModel(specs, dev)
-    workloads.init_params_into(specs, model.views(model.p), cfg + 100 * rank)
+    seed = ranks.shard_seed(cfg, rank)
+    workloads.init_params_into(specs, model.views(model.p), seed)
     sig = workloads.tensor_sigmas(specs, cfg)
-    workloads.grads_into(specs, model.views(model.g), cfg + 100 * rank, 1, sig)
+    workloads.grads_into(specs, model.views(model.g), seed, 1, sig)
     opt = FP8AdamW(model.views(model.p), model.views(model.g), m=model.views(model.m), v=model.views(model.v),
                    scale_m=model.scale_m, scale_v=model.scale_v, amax_m=model.amax_m, amax_v=model.amax_v)
     stream = torch.cuda.current_stream(dev)
@@ -259,10 +256,7 @@ def our_arm(args):
     clk = clocks.stop()
     elapsed = t_start.elapsed_time(t_end) / 1e3
     kernel_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        tt = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed = float(tt)
+    elapsed = ranks.max_over_ranks(elapsed, dev)
     value = world * n_params * args.steps / elapsed
 
     # ---- end to end: host gradients in, amax out, through the public API
@@ -282,11 +276,7 @@ def our_arm(args):
             am_host[len(specs):].copy_(model.amax_v, non_blocking=True)
         e1.record(stream)
         barrier()
-        et = e0.elapsed_time(e1) / 1e3
-        if world > 1:
-            tt = torch.tensor([et], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            et = float(tt)
+        et = ranks.max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
         e2e = {"value": world * n_params * e2e_steps / et, "unit": UNIT,
                "h2d_bytes_per_step": g_host.numel() * g_host.element_size(),
                "d2h_bytes_per_step": am_host.numel() * am_host.element_size(), "steps": e2e_steps}
@@ -322,9 +312,7 @@ def our_arm(args):
                 "e2e": e2e, "gpu_launches": launches, "clocks": clk,
                 "gb_per_s": world * BYTES_PER_PARAM * n_params * args.steps / elapsed / 1e9}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.finish()
 
 
 def main():
