@@ -18,6 +18,8 @@ ERR_UNSUPPORTED_FMT = -2
 ERR_CUDA = -3
 ERR_OOM = -4
 ERR_WRONG_DEVICE = -5
+ERR_NOALLOC_LIMIT = -6
+NOALLOC_MAX_TENSORS = 4096
 
 E4M3, E5M2, FP32 = 0, 1, 2
 FLAG_STATS = 1
@@ -67,6 +69,9 @@ def lib() -> ctypes.CDLL:
         L.fp8adam_decode.argtypes = [i32, vp, vp, i64, i32, vp]
         L.fp8adam_launch_count.restype = ctypes.c_uint64
         L.fp8adam_launch_count.argtypes = []
+        L.fp8adam_step_noalloc.restype = ctypes.c_int
+        L.fp8adam_step_noalloc.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, vp, vp, vp, vp, i32, i32, u32,
+                                           f, f, f, f, f, i64, vp]
         _lib = L
     return _lib
 
@@ -127,6 +132,16 @@ def fp8adam_launch_count() -> int:
     return int(lib().fp8adam_launch_count())
 
 
+def fp8adam_step_noalloc(tensors, num_tensors: int, scale_m: int, scale_v: int, amax_m: int, amax_v: int,
+                         m_fmt: int, v_fmt: int, flags: int, lr: float, beta1: float, beta2: float,
+                         eps: float, weight_decay: float, step: int, cuda_stream: int) -> None:
+    """The allocation-free step (see include/fp8adam.h): for callers that
+    cannot allocate device memory; uses the library's fixed scratch array."""
+    _check("fp8adam_step_noalloc", lib().fp8adam_step_noalloc(
+        tensors, num_tensors, scale_m, scale_v, amax_m, amax_v, m_fmt, v_fmt, flags, lr, beta1, beta2,
+        eps, weight_decay, step, cuda_stream))
+
+
 EXPORTED = ["fp8adam_create", "fp8adam_step", "fp8adam_get_stats", "fp8adam_reset_stats",
             "fp8adam_destroy", "fp8adam_strerror", "fp8adam_encode", "fp8adam_encode_bits_range",
-            "fp8adam_decode", "fp8adam_launch_count"]
+            "fp8adam_decode", "fp8adam_launch_count", "fp8adam_step_noalloc"]

@@ -331,6 +331,7 @@ extern "C" const char* fp8adam_strerror(int code) {
     case FP8ADAM_ERR_CUDA: return "CUDA runtime error";
     case FP8ADAM_ERR_OOM: return "device allocation failed";
     case FP8ADAM_ERR_WRONG_DEVICE: return "current device differs from the context's";
+    case FP8ADAM_ERR_NOALLOC_LIMIT: return "more tensors than the allocation-free step holds (FP8ADAM_NOALLOC_MAX_TENSORS)";
     default: return "unknown error";
   }
 }

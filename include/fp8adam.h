@@ -65,6 +65,7 @@ extern "C" {
 #define FP8ADAM_ERR_CUDA (-3)            /* a CUDA runtime call failed */
 #define FP8ADAM_ERR_OOM (-4)             /* device allocation failed in create */
 #define FP8ADAM_ERR_WRONG_DEVICE (-5)    /* current device differs from create's */
+#define FP8ADAM_ERR_NOALLOC_LIMIT (-6)   /* more tensors than fp8adam_step_noalloc holds */
 
 /* Storage format of a moment. */
 typedef enum {
@@ -147,9 +148,47 @@ int fp8adam_encode_bits_range(int32_t fmt, uint32_t first, int64_t n,
 int fp8adam_decode(int32_t fmt, const uint8_t* codes, float* out, int64_t n,
                    int32_t impl, void* cuda_stream);
 
-/* Number of kernels launched by the library on this process since load (for
- * accounting launches inside a timed region). */
+/* Number of kernels launched by fp8adam_step and the codec entry points in
+ * this process since load (for accounting launches inside a timed region). */
 uint64_t fp8adam_launch_count(void);
+
+/* ---- allocation-free step ------------------------------------------------
+ * No counterpart in the paper or the pages: this is a service for callers
+ * that cannot allocate device memory -- a custom allocator or memory-pool
+ * callback, a framework hook that must not grow the footprint, a process
+ * whose memory is reserved up front, or a runtime that forbids cudaMalloc
+ * after start-up.  fp8adam_create allocates tables and accumulators; this
+ * call allocates nothing (no cudaMalloc, no cudaFree, no allocating library
+ * routine).
+ *
+ * It performs one step exactly as fp8adam_create(...) + fp8adam_step(...)
+ * with the same arguments would (same kernels' arithmetic, same results),
+ * using as scratch one fixed device array inside the library: the tensor
+ * table, per-tensor chunk offsets, amax accumulators and completion
+ * counters for at most FP8ADAM_NOALLOC_MAX_TENSORS tensors (about 288 KiB,
+ * held by every GPU that loads the library until the process exits).
+ * The caller passes all inputs and outputs as for fp8adam_create; flags may
+ * be 0 or FP8ADAM_FLAG_JIT_EVERY_STEP (no statistics).
+ *
+ * - num_tensors > FP8ADAM_NOALLOC_MAX_TENSORS returns FP8ADAM_ERR_NOALLOC_LIMIT
+ *   with nothing queued; other argument errors as fp8adam_create/step.
+ * - The first call on a device looks up the scratch array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - Each call copies the tensor table from host memory into the scratch
+ *   (the copy waits for work already queued on cuda_stream) and clears the
+ *   accumulators, so no state carries over between calls.
+ * - Every call shares the one scratch array: calls that overlap on the GPU
+ *   (different streams, or different host threads) race and must not be
+ *   issued; serialise them on one stream from one thread.
+ * - Its kernel launches are not counted by fp8adam_launch_count. */
+#define FP8ADAM_NOALLOC_MAX_TENSORS 4096
+int fp8adam_step_noalloc(const fp8adam_tensor* tensors, int32_t num_tensors,
+                         float* scale_m, float* scale_v, float* amax_m,
+                         float* amax_v, int32_t m_fmt, int32_t v_fmt,
+                         uint32_t flags, float lr, float beta1, float beta2,
+                         float eps, float weight_decay, int64_t step,
+                         void* cuda_stream);
 
 #ifdef __cplusplus
 }
