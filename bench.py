@@ -315,6 +315,71 @@ def our_arm(args):
     ranks.finish()
 
 
+def ablation_report(args):
+    """Moment-format ablation on the Llama2-100M layout ([EXPL] "实验证据
+    (Fig. 5)"): all four (m, v) format pairs and the fp32-moment run, in
+    lockstep on the same seeded gradients.  Per mode: step throughput, the
+    per-step count of v elements flushed to zero, and the per-step max
+    |p_mode - p_fp32| (gradients are open-loop, so the difference is the
+    optimizer's own error)."""
+    import torch
+
+    from fp8_quantized_adam_b200 import FP8AdamW, build, workloads
+
+    build.build()
+    dev = torch.device("cuda", 0)
+    name = "ablation_100m"
+    specs = workloads.layout(name)
+    cfg = workloads.CFG_ID[name]
+    n_params = workloads.total_params(specs)
+    modes = {"m4v4": ("e4m3", "e4m3"), "m4v5": ("e4m3", "e5m2"), "m5v4": ("e5m2", "e4m3"),
+             "m5v5": ("e5m2", "e5m2"), "fp32": ("fp32", "fp32")}
+    models, opts = {}, {}
+    g = workloads.FlatModel(specs, dev).g  # one gradient buffer shared by all modes
+    for k, (mf, vf) in modes.items():
+        M = workloads.FlatModel(specs, dev, m_fp32=mf == "fp32", v_fp32=vf == "fp32")
+        workloads.init_params_into(specs, M.views(M.p), cfg)
+        M.g = g
+        models[k] = M
+        opts[k] = FP8AdamW(M.views(M.p), M.views(g), m_fmt=mf, v_fmt=vf, m=M.views(M.m), v=M.views(M.v),
+                           scale_m=M.scale_m, scale_v=M.scale_v, amax_m=M.amax_m, amax_v=M.amax_v,
+                           stats=True)
+    sig = workloads.tensor_sigmas(specs, cfg)
+    off = workloads.offsets(specs)
+    views = [g[off[i]:off[i] + s.numel] for i, s in enumerate(specs)]
+    out = {k: {"flushed_v": [], "saturated": [], "max_abs_dp_vs_fp32": [], "ms": []} for k in modes}
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for t in range(1, args.steps + 1):
+        workloads.grads_into(specs, views, cfg, t, sig)
+        for k in modes:
+            opts[k].reset_stats()
+            ev[0].record()
+            opts[k].step()
+            ev[1].record()
+            ev[1].synchronize()
+            out[k]["ms"].append(ev[0].elapsed_time(ev[1]))
+            f, s_ = opts[k].stats()
+            out[k]["flushed_v"].append(f)
+            out[k]["saturated"].append(s_)
+        for k in modes:
+            d = (models[k].p - models["fp32"].p).abs().max()
+            out[k]["max_abs_dp_vs_fp32"].append(float(d))
+    res = {}
+    for k, (mf, vf) in modes.items():
+        ms = sorted(out[k]["ms"][3:] or out[k]["ms"])
+        med = ms[len(ms) // 2]
+        bpp = 4 + 2 + 4 + (8 if mf == "fp32" else 2) + (8 if vf == "fp32" else 2)
+        res[k] = {"m_fmt": mf, "v_fmt": vf, "params_per_s": n_params / (med / 1e3),
+                  "gb_per_s": bpp * n_params / (med / 1e3) / 1e9, "bytes_per_param": bpp,
+                  "flushed_v_mean": sum(out[k]["flushed_v"]) / args.steps,
+                  "final_max_abs_dp_vs_fp32": out[k]["max_abs_dp_vs_fp32"][-1], **out[k]}
+        del res[k]["ms"]
+    for o in opts.values():
+        o.close()
+    print(json.dumps({"report": "format_ablation", "workload": name, "params": n_params, "steps": args.steps,
+                      "data": "synthetic", "modes": res}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -325,8 +390,12 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--report", choices=["ablation"], default=None,
+                    help="ablation: the moment-format ablation on the Llama2-100M layout")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.report == "ablation":
+        ablation_report(args)
+    elif args.impl == "reference":
         reference_arm(args)
     else:
         our_arm(args)

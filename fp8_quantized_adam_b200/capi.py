@@ -24,11 +24,27 @@ NOALLOC_MAX_TENSORS = 4096
 E4M3, E5M2, FP32 = 0, 1, 2
 FLAG_STATS = 1
 FLAG_JIT_EVERY_STEP = 2
+FLAG_UPDATE_FROM_STORED = 4
+FLAG_STOCHASTIC_ROUNDING = 8
 
 
 class fp8adam_tensor(ctypes.Structure):
     _fields_ = [("param", ctypes.c_void_p), ("grad", ctypes.c_void_p), ("m", ctypes.c_void_p),
                 ("v", ctypes.c_void_p), ("numel", ctypes.c_int64)]
+
+
+class fp8adam_options(ctypes.Structure):
+    _fields_ = [("scale_m", ctypes.c_void_p), ("scale_v", ctypes.c_void_p), ("amax_m", ctypes.c_void_p),
+                ("amax_v", ctypes.c_void_p), ("m_fmt", ctypes.c_int32), ("v_fmt", ctypes.c_int32),
+                ("flags", ctypes.c_uint32), ("margin_m", ctypes.c_int32), ("margin_v", ctypes.c_int32),
+                ("amax_history_len", ctypes.c_int32), ("amax_history_m", ctypes.c_void_p),
+                ("amax_history_v", ctypes.c_void_p), ("seed", ctypes.c_uint64), ("param_bf16", ctypes.c_void_p)]
+
+
+class fp8adam_step_params(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64),
+                ("loss_scale", ctypes.c_float), ("max_norm", ctypes.c_float), ("skip_nonfinite", ctypes.c_int32)]
 
 
 class Fp8AdamError(RuntimeError):
@@ -69,6 +85,13 @@ def lib() -> ctypes.CDLL:
         L.fp8adam_decode.argtypes = [i32, vp, vp, i64, i32, vp]
         L.fp8adam_launch_count.restype = ctypes.c_uint64
         L.fp8adam_launch_count.argtypes = []
+        L.fp8adam_create_ex.restype = ctypes.c_int
+        L.fp8adam_create_ex.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, ctypes.POINTER(fp8adam_options),
+                                        ctypes.POINTER(vp)]
+        L.fp8adam_step_ex.restype = ctypes.c_int
+        L.fp8adam_step_ex.argtypes = [vp, ctypes.POINTER(fp8adam_step_params), vp]
+        L.fp8adam_get_grad_info.restype = ctypes.c_int
+        L.fp8adam_get_grad_info.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint32), vp]
         L.fp8adam_step_noalloc.restype = ctypes.c_int
         L.fp8adam_step_noalloc.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, vp, vp, vp, vp, i32, i32, u32,
                                            f, f, f, f, f, i64, vp]
@@ -95,6 +118,23 @@ def fp8adam_create(tensors, num_tensors: int, scale_m: int, scale_v: int, amax_m
     _check("fp8adam_create", lib().fp8adam_create(tensors, num_tensors, scale_m, scale_v, amax_m, amax_v,
                                                   m_fmt, v_fmt, flags, ctypes.byref(out)))
     return out.value
+
+
+def fp8adam_create_ex(tensors, num_tensors: int, opts: fp8adam_options) -> int:
+    out = ctypes.c_void_p()
+    _check("fp8adam_create_ex", lib().fp8adam_create_ex(tensors, num_tensors, ctypes.byref(opts), ctypes.byref(out)))
+    return out.value
+
+
+def fp8adam_step_ex(ctx: int, params: fp8adam_step_params, cuda_stream: int) -> None:
+    _check("fp8adam_step_ex", lib().fp8adam_step_ex(ctx, ctypes.byref(params), cuda_stream))
+
+
+def fp8adam_get_grad_info(ctx: int, cuda_stream: int):
+    n = ctypes.c_double()
+    k = ctypes.c_uint32()
+    _check("fp8adam_get_grad_info", lib().fp8adam_get_grad_info(ctx, ctypes.byref(n), ctypes.byref(k), cuda_stream))
+    return n.value, int(k.value)
 
 
 def fp8adam_step(ctx: int, lr: float, beta1: float, beta2: float, eps: float, weight_decay: float,
@@ -144,4 +184,5 @@ def fp8adam_step_noalloc(tensors, num_tensors: int, scale_m: int, scale_v: int, 
 
 EXPORTED = ["fp8adam_create", "fp8adam_step", "fp8adam_get_stats", "fp8adam_reset_stats",
             "fp8adam_destroy", "fp8adam_strerror", "fp8adam_encode", "fp8adam_encode_bits_range",
-            "fp8adam_decode", "fp8adam_launch_count", "fp8adam_step_noalloc"]
+            "fp8adam_decode", "fp8adam_launch_count", "fp8adam_step_noalloc", "fp8adam_create_ex",
+            "fp8adam_step_ex", "fp8adam_get_grad_info"]

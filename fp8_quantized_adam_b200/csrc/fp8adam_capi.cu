@@ -1,8 +1,9 @@
 // fp8adam_capi.cu -- the C ABI declared in include/fp8adam.h.
 //
 // Host side of the FP8-moment AdamW step: argument validation, the device
-// tensor/chunk tables, per-step constants (computed in double, rounded once
-// to fp32) and kernel dispatch over the (m format, v format, stats) variants.
+// tensor table and tile prefix, persistent grid sizing, per-step constants
+// (computed in double, rounded once to fp32) and kernel dispatch over the
+// (m format, v format, stats) variants.
 // The kernels are in fp8adam_step.cuh; the codec in fp8_codec.cuh.
 
 #include <cuda_runtime.h>
@@ -16,6 +17,7 @@
 
 #include "../../include/fp8adam.h"
 #include "fp8_codec.cuh"
+#include "fp8adam_ext.cuh"
 #include "fp8adam_step.cuh"
 
 using namespace fp8adam;
@@ -125,6 +127,27 @@ StepFn pick_amax(int mf, int vf) {
   return t[mf][vf];
 }
 
+using ExtFn = void (*)(const ExtArgs);
+template <int MF, int VF, bool S> ExtFn ext_fn() { return &fp8adam_step_ext_kernel<MF, VF, S>; }
+template <int MF, int VF> ExtFn aext_fn() { return &fp8adam_amax_ext_kernel<MF, VF>; }
+
+ExtFn pick_ext(int mf, int vf, bool stats) {
+  static const ExtFn t[3][3][2] = {
+      {{ext_fn<0, 0, false>(), ext_fn<0, 0, true>()}, {ext_fn<0, 1, false>(), ext_fn<0, 1, true>()},
+       {ext_fn<0, 2, false>(), ext_fn<0, 2, true>()}},
+      {{ext_fn<1, 0, false>(), ext_fn<1, 0, true>()}, {ext_fn<1, 1, false>(), ext_fn<1, 1, true>()},
+       {ext_fn<1, 2, false>(), ext_fn<1, 2, true>()}},
+      {{ext_fn<2, 0, false>(), ext_fn<2, 0, true>()}, {ext_fn<2, 1, false>(), ext_fn<2, 1, true>()},
+       {ext_fn<2, 2, false>(), ext_fn<2, 2, true>()}}};
+  return t[mf][vf][stats ? 1 : 0];
+}
+ExtFn pick_amax_ext(int mf, int vf) {
+  static const ExtFn t[3][3] = {{aext_fn<0, 0>(), aext_fn<0, 1>(), aext_fn<0, 2>()},
+                                {aext_fn<1, 0>(), aext_fn<1, 1>(), aext_fn<1, 2>()},
+                                {aext_fn<2, 0>(), aext_fn<2, 1>(), aext_fn<2, 2>()}};
+  return t[mf][vf];
+}
+
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 }  // namespace
@@ -135,10 +158,27 @@ struct fp8adam_ctx {
   int32_t T = 0;
   int32_t m_fmt = 0, v_fmt = 0;
   uint32_t flags = 0;
-  int32_t nchunks = 0;
+  int32_t total_units = 0;                        // work units of the schedule
+  int32_t step_grid = 0, step_tiles_per_cta = 0;  // grid of the step kernel
+  int32_t amax_grid = 0, amax_tiles_per_cta = 0;  // and of the pre-pass
   float *scale_m = nullptr, *scale_v = nullptr, *amax_m = nullptr, *amax_v = nullptr;
   TensorDesc* d_tensors = nullptr;
-  Chunk* d_chunks = nullptr;
+  int32_t* d_unit_begin = nullptr;
+  Chunk* d_chunks = nullptr;  // chunk schedule
+  // options of fp8adam_create_ex
+  int32_t margin_m = 0, margin_v = 0, hist_len = 0;
+  float *hist_m = nullptr, *hist_v = nullptr;
+  uint64_t seed = 0;
+  uint16_t** d_bf16 = nullptr;  // device [T] bf16 outputs, or null
+  bool ext = false;             // any option on: the variant kernels run
+  int32_t ext_grid = 0, ext_tiles_per_cta = 0, aext_grid = 0, aext_tiles_per_cta = 0;
+  // gradient pre-pass of fp8adam_step_ex: [step_grid] partials, non-finite
+  // count, multiplier, skip flag, norm
+  double* d_partial = nullptr;
+  unsigned long long* d_nonfinite = nullptr;
+  float* d_grad_mult = nullptr;
+  uint32_t* d_skip = nullptr;
+  double* d_norm = nullptr;
   uint32_t* d_state = nullptr;  // [5T]: acc_m, acc_v, jit_m, jit_v, done
   unsigned long long* d_stats = nullptr;
 };
@@ -146,10 +186,41 @@ struct fp8adam_ctx {
 static void free_ctx(fp8adam_ctx* c) {
   if (!c) return;
   cudaFree(c->d_tensors);
+  cudaFree(c->d_unit_begin);
   cudaFree(c->d_chunks);
+  cudaFree(c->d_bf16);
+  cudaFree(c->d_partial);
+  cudaFree(c->d_nonfinite);
+  cudaFree(c->d_grad_mult);
+  cudaFree(c->d_skip);
+  cudaFree(c->d_norm);
   cudaFree(c->d_state);
   cudaFree(c->d_stats);
   delete c;
+}
+
+// Grid of a kernel over the context's work units.  One CTA per chunk, or
+// (persistent schedule) every SM filled with as many CTAs as can be resident,
+// each taking a contiguous, equal range of tiles (no CTA without work).
+static int size_grid(const fp8adam_ctx* c, const void* kernel, int32_t* grid, int32_t* per_cta) {
+#if !FP8ADAM_PERSISTENT
+  (void)kernel;
+  *grid = c->total_units > 0 ? c->total_units : 1;
+  *per_cta = 1;
+  return FP8ADAM_OK;
+#endif
+  int sms = 0, occ = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, 0) != cudaSuccess) {
+    cudaGetLastError();
+    return FP8ADAM_ERR_CUDA;
+  }
+  const int64_t slots = (int64_t)sms * (occ > 0 ? occ : 1);
+  const int64_t tiles = c->total_units > 0 ? c->total_units : 1;
+  const int64_t per = (tiles + slots - 1) / slots;
+  *per_cta = (int32_t)per;
+  *grid = (int32_t)((tiles + per - 1) / per);
+  return FP8ADAM_OK;
 }
 
 extern "C" int fp8adam_create(const fp8adam_tensor* tensors, int32_t num_tensors, float* scale_m,
@@ -157,42 +228,65 @@ extern "C" int fp8adam_create(const fp8adam_tensor* tensors, int32_t num_tensors
                               int32_t v_fmt, uint32_t flags, fp8adam_ctx** out) {
   if (!out) return FP8ADAM_ERR_INVALID_ARG;
   *out = nullptr;
+  if (flags & ~(FP8ADAM_FLAG_STATS | FP8ADAM_FLAG_JIT_EVERY_STEP)) return FP8ADAM_ERR_INVALID_ARG;
+  fp8adam_options o;
+  std::memset(&o, 0, sizeof(o));
+  o.scale_m = scale_m;
+  o.scale_v = scale_v;
+  o.amax_m = amax_m;
+  o.amax_v = amax_v;
+  o.m_fmt = m_fmt;
+  o.v_fmt = v_fmt;
+  o.flags = flags;
+  return fp8adam_create_ex(tensors, num_tensors, &o, out);
+}
+
+extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tensors, const fp8adam_options* opts,
+                                 fp8adam_ctx** out) {
+  if (!out) return FP8ADAM_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!opts) return FP8ADAM_ERR_INVALID_ARG;
+  float *scale_m = opts->scale_m, *scale_v = opts->scale_v, *amax_m = opts->amax_m, *amax_v = opts->amax_v;
+  const int32_t m_fmt = opts->m_fmt, v_fmt = opts->v_fmt;
+  const uint32_t flags = opts->flags;
   if (!tensors || num_tensors < 1 || !scale_m || !scale_v || !amax_m || !amax_v)
     return FP8ADAM_ERR_INVALID_ARG;
   if (m_fmt < 0 || m_fmt > 2 || v_fmt < 0 || v_fmt > 2) return FP8ADAM_ERR_UNSUPPORTED_FMT;
-  if (flags & ~(FP8ADAM_FLAG_STATS | FP8ADAM_FLAG_JIT_EVERY_STEP)) return FP8ADAM_ERR_INVALID_ARG;
+  if (flags & ~(FP8ADAM_FLAG_STATS | FP8ADAM_FLAG_JIT_EVERY_STEP | FP8ADAM_FLAG_UPDATE_FROM_STORED |
+                FP8ADAM_FLAG_STOCHASTIC_ROUNDING))
+    return FP8ADAM_ERR_INVALID_ARG;
+  if (opts->margin_m < 0 || opts->margin_m > 64 || opts->margin_v < 0 || opts->margin_v > 64 ||
+      opts->amax_history_len < 0 || opts->amax_history_len > 1024 ||
+      (opts->amax_history_len > 1 && (!opts->amax_history_m || !opts->amax_history_v)))
+    return FP8ADAM_ERR_INVALID_ARG;
 
   std::vector<TensorDesc> desc((size_t)num_tensors);
-  std::vector<Chunk> chunks;
-  int64_t total_chunks = 0;
+  std::vector<int32_t> unit_begin((size_t)num_tensors + 1);
+  int64_t total_units = 0;
   for (int32_t i = 0; i < num_tensors; ++i) {
     const fp8adam_tensor& t = tensors[i];
     if (t.numel < 0) return FP8ADAM_ERR_INVALID_ARG;
     if (t.numel > 0 && (!t.param || !t.grad || !t.m || !t.v)) return FP8ADAM_ERR_INVALID_ARG;
-    const int64_t nc = (t.numel + kChunk - 1) / kChunk;
-    if (nc > INT32_MAX) return FP8ADAM_ERR_INVALID_ARG;
-    total_chunks += nc;
-  }
-  if (total_chunks > INT32_MAX) return FP8ADAM_ERR_INVALID_ARG;
-  chunks.reserve((size_t)total_chunks);
-  for (int32_t i = 0; i < num_tensors; ++i) {
-    const fp8adam_tensor& t = tensors[i];
+    const int64_t nt = (t.numel + kUnit - 1) / kUnit;
+    unit_begin[(size_t)i] = (int32_t)total_units;
+    total_units += nt;
+    if (total_units > INT32_MAX / 2) return FP8ADAM_ERR_INVALID_ARG;
     TensorDesc& d = desc[(size_t)i];
     d.p = t.param;
     d.g = t.grad;
     d.m = t.m;
     d.v = t.v;
     d.numel = t.numel;
-    d.nchunks = (int32_t)((t.numel + kChunk - 1) / kChunk);
+    d.nunits = (int32_t)nt;
     d.aligned = aligned16(t.param) && aligned16(t.grad) && aligned16(t.m) && aligned16(t.v);
-    for (int64_t s = 0; s < t.numel; s += kChunk) {
-      Chunk c;
-      c.tensor = i;
-      c.start = s;
-      c.len = (int32_t)(t.numel - s < kChunk ? t.numel - s : kChunk);
-      chunks.push_back(c);
-    }
   }
+  unit_begin[(size_t)num_tensors] = (int32_t)total_units;
+  std::vector<Chunk> chunks;
+#if !FP8ADAM_PERSISTENT
+  chunks.reserve((size_t)total_units);
+  for (int32_t i = 0; i < num_tensors; ++i)
+    for (int64_t st = 0; st < tensors[i].numel; st += kChunk) chunks.push_back(Chunk{i, 0, st});
+#endif
 
   fp8adam_ctx* c = new (std::nothrow) fp8adam_ctx();
   if (!c) return FP8ADAM_ERR_OOM;
@@ -204,13 +298,22 @@ extern "C" int fp8adam_create(const fp8adam_tensor* tensors, int32_t num_tensors
   c->m_fmt = m_fmt;
   c->v_fmt = v_fmt;
   c->flags = flags;
-  c->nchunks = (int32_t)chunks.size();
+  c->total_units = (int32_t)total_units;
   c->scale_m = scale_m;
   c->scale_v = scale_v;
   c->amax_m = amax_m;
   c->amax_v = amax_v;
+  c->margin_m = opts->margin_m;
+  c->margin_v = opts->margin_v;
+  c->hist_len = opts->amax_history_len > 1 ? opts->amax_history_len : 0;
+  c->hist_m = c->hist_len ? opts->amax_history_m : nullptr;
+  c->hist_v = c->hist_len ? opts->amax_history_v : nullptr;
+  c->seed = opts->seed;
+  c->ext = (flags & (FP8ADAM_FLAG_UPDATE_FROM_STORED | FP8ADAM_FLAG_STOCHASTIC_ROUNDING)) || c->margin_m ||
+           c->margin_v || c->hist_len || opts->param_bf16;
   const size_t T = (size_t)num_tensors;
   if (cudaMalloc(&c->d_tensors, T * sizeof(TensorDesc)) != cudaSuccess ||
+      cudaMalloc(&c->d_unit_begin, (T + 1) * sizeof(int32_t)) != cudaSuccess ||
       cudaMalloc(&c->d_chunks, (chunks.empty() ? 1 : chunks.size()) * sizeof(Chunk)) != cudaSuccess ||
       cudaMalloc(&c->d_state, 5 * T * sizeof(uint32_t)) != cudaSuccess ||
       cudaMalloc(&c->d_stats, 2 * sizeof(unsigned long long)) != cudaSuccess) {
@@ -219,11 +322,43 @@ extern "C" int fp8adam_create(const fp8adam_tensor* tensors, int32_t num_tensors
     return FP8ADAM_ERR_OOM;
   }
   if (cudaMemcpy(c->d_tensors, desc.data(), T * sizeof(TensorDesc), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(c->d_unit_begin, unit_begin.data(), (T + 1) * sizeof(int32_t), cudaMemcpyHostToDevice) !=
+          cudaSuccess ||
       (!chunks.empty() &&
-       cudaMemcpy(c->d_chunks, chunks.data(), chunks.size() * sizeof(Chunk), cudaMemcpyHostToDevice) !=
-           cudaSuccess) ||
+       cudaMemcpy(c->d_chunks, chunks.data(), chunks.size() * sizeof(Chunk), cudaMemcpyHostToDevice) != cudaSuccess) ||
       cudaMemset(c->d_state, 0, 5 * T * sizeof(uint32_t)) != cudaSuccess ||
       cudaMemset(c->d_stats, 0, 2 * sizeof(unsigned long long)) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    free_ctx(c);
+    return FP8ADAM_ERR_CUDA;
+  }
+  const bool stats = (flags & FP8ADAM_FLAG_STATS) != 0;
+  if (size_grid(c, (const void*)pick_step(m_fmt, v_fmt, stats), &c->step_grid, &c->step_tiles_per_cta) !=
+          FP8ADAM_OK ||
+      size_grid(c, (const void*)pick_amax(m_fmt, v_fmt), &c->amax_grid, &c->amax_tiles_per_cta) != FP8ADAM_OK ||
+      size_grid(c, (const void*)pick_ext(m_fmt, v_fmt, stats), &c->ext_grid, &c->ext_tiles_per_cta) !=
+          FP8ADAM_OK ||
+      size_grid(c, (const void*)pick_amax_ext(m_fmt, v_fmt), &c->aext_grid, &c->aext_tiles_per_cta) !=
+          FP8ADAM_OK) {
+    free_ctx(c);
+    return FP8ADAM_ERR_CUDA;
+  }
+  // gradient pre-pass buffers (partials over the step grid) and options
+  if (cudaMalloc(&c->d_partial, (size_t)(c->step_grid > 0 ? c->step_grid : 1) * sizeof(double)) != cudaSuccess ||
+      cudaMalloc(&c->d_nonfinite, sizeof(unsigned long long)) != cudaSuccess ||
+      cudaMalloc(&c->d_grad_mult, sizeof(float)) != cudaSuccess ||
+      cudaMalloc(&c->d_skip, sizeof(uint32_t)) != cudaSuccess ||
+      cudaMalloc(&c->d_norm, sizeof(double)) != cudaSuccess ||
+      (opts->param_bf16 && cudaMalloc(&c->d_bf16, T * sizeof(uint16_t*)) != cudaSuccess)) {
+    cudaGetLastError();
+    free_ctx(c);
+    return FP8ADAM_ERR_OOM;
+  }
+  if (cudaMemset(c->d_skip, 0, sizeof(uint32_t)) != cudaSuccess ||
+      cudaMemset(c->d_norm, 0, sizeof(double)) != cudaSuccess ||
+      (opts->param_bf16 &&
+       cudaMemcpy(c->d_bf16, opts->param_bf16, T * sizeof(uint16_t*), cudaMemcpyHostToDevice) != cudaSuccess) ||
       cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     free_ctx(c);
@@ -233,30 +368,31 @@ extern "C" int fp8adam_create(const fp8adam_tensor* tensors, int32_t num_tensors
   return FP8ADAM_OK;
 }
 
-extern "C" int fp8adam_step(fp8adam_ctx* ctx, float lr, float beta1, float beta2, float eps,
-                            float weight_decay, int64_t step, void* cuda_stream) {
-  if (!ctx) return FP8ADAM_ERR_INVALID_ARG;
-  if (step < 1 || !std::isfinite(lr) || !std::isfinite(weight_decay) || !(beta1 >= 0.0f) ||
-      !(beta1 < 1.0f) || !(beta2 >= 0.0f) || !(beta2 < 1.0f) || !(eps >= 0.0f) || !std::isfinite(eps))
-    return FP8ADAM_ERR_INVALID_ARG;
+static bool valid_hparams(float lr, float beta1, float beta2, float eps, float weight_decay, int64_t step) {
+  return step >= 1 && std::isfinite(lr) && std::isfinite(weight_decay) && beta1 >= 0.0f && beta1 < 1.0f &&
+         beta2 >= 0.0f && beta2 < 1.0f && eps >= 0.0f && std::isfinite(eps);
+}
+
+static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t st) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return FP8ADAM_ERR_CUDA;
   if (dev != ctx->device) return FP8ADAM_ERR_WRONG_DEVICE;
-  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  if (ctx->nchunks == 0) return FP8ADAM_OK;  // every tensor empty
+  if (ctx->total_units == 0) return FP8ADAM_OK;  // every tensor empty
+  const bool prepass = p.loss_scale != 1.0f || p.max_norm > 0.0f || p.skip_nonfinite != 0;
+  const bool ext = ctx->ext || prepass;
 
   // constants of step t: double, rounded once to fp32
-  const double bc1 = 1.0 - std::pow((double)beta1, (double)step);
-  const double bc2 = 1.0 - std::pow((double)beta2, (double)step);
+  const double bc1 = 1.0 - std::pow((double)p.beta1, (double)p.step);
+  const double bc2 = 1.0 - std::pow((double)p.beta2, (double)p.step);
   StepArgs a;
-  a.c.b1 = beta1;
-  a.c.omb1 = (float)(1.0 - (double)beta1);
-  a.c.b2 = beta2;
-  a.c.omb2 = (float)(1.0 - (double)beta2);
-  a.c.step_size = (float)((double)lr / bc1);
+  a.c.b1 = p.beta1;
+  a.c.omb1 = (float)(1.0 - (double)p.beta1);
+  a.c.b2 = p.beta2;
+  a.c.omb2 = (float)(1.0 - (double)p.beta2);
+  a.c.step_size = (float)((double)p.lr / bc1);
   a.c.isbc2 = (float)(1.0 / std::sqrt(bc2));
-  a.c.eps = eps;
-  a.c.decay = (float)(1.0 - (double)lr * (double)weight_decay);
+  a.c.eps = p.eps;
+  a.c.decay = (float)(1.0 - (double)p.lr * (double)p.weight_decay);
 
   const size_t T = (size_t)ctx->T;
   uint32_t* acc_m = ctx->d_state;
@@ -264,24 +400,84 @@ extern "C" int fp8adam_step(fp8adam_ctx* ctx, float lr, float beta1, float beta2
   uint32_t* jit_m = ctx->d_state + 2 * T;
   uint32_t* jit_v = ctx->d_state + 3 * T;
   a.tensors = ctx->d_tensors;
+  a.unit_begin = ctx->d_unit_begin;
   a.chunks = ctx->d_chunks;
+  a.num_tensors = ctx->T;
+  a.total_tiles = ctx->total_units;
   a.scale_m = ctx->scale_m;
   a.scale_v = ctx->scale_v;
   a.amax_m = ctx->amax_m;
   a.amax_v = ctx->amax_v;
   a.done = ctx->d_state + 4 * T;
   a.stats = ctx->d_stats;
+  a.acc_m = acc_m;
+  a.acc_v = acc_v;
 
-  const dim3 grid((unsigned)ctx->nchunks), block(kThreads);
-  const bool jit = step == 1 || (ctx->flags & FP8ADAM_FLAG_JIT_EVERY_STEP);
+  const dim3 block(kThreads);
+  const bool jit = p.step == 1 || (ctx->flags & FP8ADAM_FLAG_JIT_EVERY_STEP);
+  const bool stats = (ctx->flags & FP8ADAM_FLAG_STATS) != 0;
+  if (!ext) {
+    if (jit) {
+      if (cudaMemsetAsync(jit_m, 0, 2 * T * sizeof(uint32_t), st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
+      StepArgs pre = a;
+      pre.acc_m = jit_m;
+      pre.acc_v = jit_v;
+      pre.amax_in_m = nullptr;
+      pre.amax_in_v = nullptr;
+      pre.tiles_per_cta = ctx->amax_tiles_per_cta;
+      pick_amax(ctx->m_fmt, ctx->v_fmt)<<<dim3((unsigned)ctx->amax_grid), block, 0, st>>>(pre);
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      a.amax_in_m = jit_m;
+      a.amax_in_v = jit_v;
+    } else {
+      a.amax_in_m = reinterpret_cast<const uint32_t*>(ctx->amax_m);
+      a.amax_in_v = reinterpret_cast<const uint32_t*>(ctx->amax_v);
+    }
+    a.tiles_per_cta = ctx->step_tiles_per_cta;
+    pick_step(ctx->m_fmt, ctx->v_fmt, stats)<<<dim3((unsigned)ctx->step_grid), block, 0, st>>>(a);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return last_error();
+  }
+
+  ExtArgs e;
+  e.flags = ctx->flags & (FP8ADAM_FLAG_UPDATE_FROM_STORED | FP8ADAM_FLAG_STOCHASTIC_ROUNDING);
+  e.margin_m = ctx->margin_m;
+  e.margin_v = ctx->margin_v;
+  e.use_hist = (ctx->hist_len > 1 && !jit) ? 1 : 0;
+  e.hist_len = ctx->hist_len;
+  e.hist_slot = ctx->hist_len ? (int32_t)((p.step - 1) % ctx->hist_len) : 0;
+  e.hist_m = ctx->hist_m;
+  e.hist_v = ctx->hist_v;
+  e.seed_lo = (uint32_t)ctx->seed;
+  e.seed_hi = (uint32_t)(ctx->seed >> 32);
+  e.t_lo = (uint32_t)p.step;
+  e.grad_mult = nullptr;
+  e.skip = nullptr;
+  e.p_bf16 = ctx->d_bf16;
+  if (prepass) {
+    StepArgs g = a;
+    g.tiles_per_cta = ctx->step_tiles_per_cta;
+    if (cudaMemsetAsync(ctx->d_nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)
+      return FP8ADAM_ERR_CUDA;
+    fp8adam_gradnorm_partial_kernel<<<dim3((unsigned)ctx->step_grid), block, 0, st>>>(g, ctx->d_partial,
+                                                                                      ctx->d_nonfinite);
+    fp8adam_gradnorm_finalize_kernel<<<1, block, 0, st>>>(ctx->d_partial, ctx->step_grid, ctx->d_nonfinite,
+                                                          p.loss_scale, p.max_norm, p.skip_nonfinite,
+                                                          ctx->d_grad_mult, ctx->d_skip, ctx->d_norm);
+    g_launches.fetch_add(2, std::memory_order_relaxed);
+    e.grad_mult = ctx->d_grad_mult;
+    e.skip = ctx->d_skip;
+  }
   if (jit) {
     if (cudaMemsetAsync(jit_m, 0, 2 * T * sizeof(uint32_t), st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
-    StepArgs pre = a;
-    pre.acc_m = jit_m;
-    pre.acc_v = jit_v;
-    pre.amax_in_m = nullptr;
-    pre.amax_in_v = nullptr;
-    pick_amax(ctx->m_fmt, ctx->v_fmt)<<<grid, block, 0, st>>>(pre);
+    ExtArgs pre = e;
+    pre.s = a;
+    pre.s.acc_m = jit_m;
+    pre.s.acc_v = jit_v;
+    pre.s.amax_in_m = nullptr;
+    pre.s.amax_in_v = nullptr;
+    pre.s.tiles_per_cta = ctx->aext_tiles_per_cta;
+    pick_amax_ext(ctx->m_fmt, ctx->v_fmt)<<<dim3((unsigned)ctx->aext_grid), block, 0, st>>>(pre);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     a.amax_in_m = jit_m;
     a.amax_in_v = jit_v;
@@ -289,11 +485,52 @@ extern "C" int fp8adam_step(fp8adam_ctx* ctx, float lr, float beta1, float beta2
     a.amax_in_m = reinterpret_cast<const uint32_t*>(ctx->amax_m);
     a.amax_in_v = reinterpret_cast<const uint32_t*>(ctx->amax_v);
   }
-  a.acc_m = acc_m;
-  a.acc_v = acc_v;
-  pick_step(ctx->m_fmt, ctx->v_fmt, (ctx->flags & FP8ADAM_FLAG_STATS) != 0)<<<grid, block, 0, st>>>(a);
+  a.tiles_per_cta = ctx->ext_tiles_per_cta;
+  e.s = a;
+  pick_ext(ctx->m_fmt, ctx->v_fmt, stats)<<<dim3((unsigned)ctx->ext_grid), block, 0, st>>>(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return last_error();
+}
+
+extern "C" int fp8adam_step(fp8adam_ctx* ctx, float lr, float beta1, float beta2, float eps,
+                            float weight_decay, int64_t step, void* cuda_stream) {
+  if (!ctx) return FP8ADAM_ERR_INVALID_ARG;
+  if (!valid_hparams(lr, beta1, beta2, eps, weight_decay, step)) return FP8ADAM_ERR_INVALID_ARG;
+  fp8adam_step_params p;
+  p.lr = lr;
+  p.beta1 = beta1;
+  p.beta2 = beta2;
+  p.eps = eps;
+  p.weight_decay = weight_decay;
+  p.step = step;
+  p.loss_scale = 1.0f;
+  p.max_norm = 0.0f;
+  p.skip_nonfinite = 0;
+  return run_step(ctx, p, static_cast<cudaStream_t>(cuda_stream));
+}
+
+extern "C" int fp8adam_step_ex(fp8adam_ctx* ctx, const fp8adam_step_params* params, void* cuda_stream) {
+  if (!ctx || !params) return FP8ADAM_ERR_INVALID_ARG;
+  const fp8adam_step_params& p = *params;
+  if (!valid_hparams(p.lr, p.beta1, p.beta2, p.eps, p.weight_decay, p.step)) return FP8ADAM_ERR_INVALID_ARG;
+  if (!(p.loss_scale > 0.0f) || !std::isfinite(p.loss_scale) || std::isnan(p.max_norm) ||
+      std::isinf(p.max_norm))
+    return FP8ADAM_ERR_INVALID_ARG;
+  return run_step(ctx, p, static_cast<cudaStream_t>(cuda_stream));
+}
+
+extern "C" int fp8adam_get_grad_info(fp8adam_ctx* ctx, double* grad_norm, uint32_t* skipped, void* cuda_stream) {
+  if (!ctx || !grad_norm || !skipped) return FP8ADAM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  double n = 0.0;
+  uint32_t k = 0;
+  if (cudaMemcpyAsync(&n, ctx->d_norm, sizeof(double), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(&k, ctx->d_skip, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return FP8ADAM_ERR_CUDA;
+  *grad_norm = n;
+  *skipped = k;
+  return FP8ADAM_OK;
 }
 
 extern "C" int fp8adam_get_stats(fp8adam_ctx* ctx, uint64_t* out, void* cuda_stream) {

@@ -1,0 +1,423 @@
+// fp8adam_ext.cuh -- optional variants of the FP8-moment AdamW step.
+//
+// These are the options of fp8adam_create_ex / fp8adam_step_ex; the default
+// step (fp8adam_step_kernel) contains none of them.
+//   - amax history (DelayedScaling "amax_history_len", algo MAX) and margin
+//     ("margin"), from the transformer_engine example of "FP8训练的稳定性挑战…";
+//   - update from the stored (requantised) moments instead of this step's
+//     fp32 ones (the reading behind the daoxuan.cc explainer's "1/(0+eps)"
+//     case, sub-section "一个数值例子");
+//   - stochastic rounding of the codes ("随机舍入" in "应对FP8训练稳定性挑战的
+//     策略"), with random bits from Philox4x32-10 (Salmon, Moraes, Dror, Shaw,
+//     "Parallel random numbers: as easy as 1, 2, 3", SC 2011);
+//   - a fused gradient multiplier (loss-scale removal and global-norm
+//     clipping: "梯度缩放", "梯度裁剪" and the clip_grad_norm_ example) and
+//     skip-on-non-finite, fed by a deterministic grad-norm pre-pass;
+//   - a bf16 copy of the updated params.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "fp8_codec.cuh"
+#include "fp8adam_step.cuh"
+
+namespace fp8adam {
+
+enum ExtFlags : uint32_t {
+  kExtFromStored = 4u,  // the update reads dec(code)/scale
+  kExtStochastic = 8u,  // stochastic rounding of the codes
+};
+
+struct ExtArgs {
+  StepArgs s;               // tensors, tiles, scales, amax, accumulators, constants
+  uint32_t flags;           // kExt* bits
+  int32_t margin_m, margin_v;
+  int32_t use_hist;         // scale from the max of the amax ring (not at JIT steps)
+  int32_t hist_len;         // ring length (>= 1 when hist_m is set)
+  int32_t hist_slot;        // this step's slot, (t-1) % hist_len
+  float* hist_m;            // [hist_len][T] or null
+  float* hist_v;
+  uint32_t seed_lo, seed_hi, t_lo;
+  const float* grad_mult;   // device scalar, or null (1.0)
+  const uint32_t* skip;     // device flag, or null
+  uint16_t* const* p_bf16;  // device array [T] of bf16 outputs (entries may be null), or null
+};
+
+// ------------------------------------------------------------ Philox4x32-10
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = 0xD2511F53u * c.x;
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// random words of elements (2q, 2q+1) of tensor ti at this step:
+// .x/.y -> element 2q (m, v); .z/.w -> element 2q+1 (m, v)
+__device__ __forceinline__ uint4 sr_words(const ExtArgs& a, int ti, int64_t q) {
+  return philox4x32_10(make_uint4((uint32_t)q, (uint32_t)((uint64_t)q >> 32), (uint32_t)ti, a.t_lo), a.seed_lo,
+                       a.seed_hi);
+}
+
+// ------------------------------------------------------------ SR encoder
+// Round up to the next grid value iff r < (|x| - lo) / (hi - lo) * 2^32 (that
+// is r * (hi - lo) < (|x| - lo) * 2^32); saturate; NaN -> 0x7F.
+template <int FMT>
+__device__ __forceinline__ uint32_t enc1_sr(float x, uint32_t r) {
+  using T = FmtTraits<FMT>;
+  const uint32_t u = __float_as_uint(x);
+  const uint32_t sign = (u >> 24) & 0x80u;
+  const uint32_t a = u & 0x7FFFFFFFu;
+  if (a > 0x7F800000u) return 0x7Fu;
+  if (a >= T::kMaxBits) return sign | T::kMaxCode;
+  const uint32_t min_normal = (uint32_t)(127 + 1 - T::kBias) << 23;
+  uint32_t code;
+  if (a < min_normal) {
+    // y = |x| / (quantum 2^(1-bias-M)), exact; n = floor(y), f = y - n exact
+    const float y = __fmul_rn(__uint_as_float(a), __uint_as_float((uint32_t)(127 + T::kBias - 1 + T::kMant) << 23));
+    const float n = floorf(y);
+    const float f = __fsub_rn(y, n);
+    const uint32_t thr = __float2uint_ru(__fmul_rn(f, 4294967296.0f));  // ceil(f * 2^32); the product is exact
+    code = (uint32_t)n + (r < thr ? 1u : 0u);
+  } else {
+    // quantum = 2^sh fp32 ulps: keep the truncated bits, round up iff the
+    // top (32 - sh) bits of r are below the dropped bits
+    constexpr int sh = 23 - T::kMant;
+    const uint32_t dropped = a & ((1u << sh) - 1u);
+    code = (a >> sh) + ((r >> (32 - sh)) < dropped ? 1u : 0u) - ((uint32_t)(127 - T::kBias) << T::kMant);
+  }
+  return sign | code;
+}
+
+// ------------------------------------------------------------ scale with margin
+template <int FMT>
+__device__ __forceinline__ float pow2scale_margin(float amax, float s_prev, int margin) {
+  const uint32_t b = __float_as_uint(amax);
+  if (!(amax > 0.0f) || b >= 0x7F800000u) return s_prev;
+  int k;
+  if (b < 0x00800000u) {
+    // subnormal amax = man * 2^-149: leading bit p gives the exponent p - 149
+    const int p = 31 - __clz(b);
+    const uint32_t frac = (b << (23 - p)) & 0x7FFFFFu;
+    k = FmtTraits<FMT>::kEmax - (p - 149) - (frac > 0x600000u ? 1 : 0);
+  } else {
+    const int e = (int)(b >> 23) - 127;
+    k = FmtTraits<FMT>::kEmax - e - ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  }
+  k -= margin;
+  k = k > 126 ? 126 : (k < -126 ? -126 : k);
+  return __uint_as_float((uint32_t)(k + 127) << 23);
+}
+
+// ------------------------------------------------------------ encode/store
+// Encodes one moment value (x * s) and returns the value the update reads.
+template <int FMT, bool STATS, bool IS_V>
+__device__ __forceinline__ float ext_q(const ExtArgs& a, float x, float s, float inv_s, uint32_t r, uint32_t& code,
+                                       uint32_t& flushed, uint32_t& sat) {
+  if constexpr (FMT == kFP32) {
+    code = 0;
+    return x;
+  } else {
+    const float y = __fmul_rn(x, s);
+    code = (a.flags & kExtStochastic) ? enc1_sr<FMT>(y, r) : enc1_hw<FMT>(y);
+    if constexpr (STATS) {
+      sat += fabsf(y) > FmtTraits<FMT>::kMax ? 1u : 0u;
+      if constexpr (IS_V) flushed += (x > 0.0f && (code & 0x7Fu) == 0u) ? 1u : 0u;
+    }
+    return (a.flags & kExtFromStored) ? __fmul_rn(dec1_hw<FMT>(code), inv_s) : x;
+  }
+}
+
+struct ExtSeg {  // per tensor segment
+  float inv_s_m, inv_s_v, s_m_new, s_v_new, inv_s_m_new, inv_s_v_new, gm;
+  uint16_t* pb;
+  int ti;
+};
+
+// One element (tails, unaligned tensors).
+template <int MF, int VF, bool STATS>
+__device__ __forceinline__ void ext_element(const ExtArgs& a, const TensorDesc& td, const ExtSeg& sg, int64_t i,
+                                            float& am, float& av, uint32_t& flushed, uint32_t& sat) {
+  const StepConsts& c = a.s.c;
+  uint32_t rm = 0, rv = 0;
+  if (a.flags & kExtStochastic) {
+    const uint4 r = sr_words(a, sg.ti, i >> 1);
+    rm = (i & 1) ? r.z : r.x;
+    rv = (i & 1) ? r.w : r.y;
+  }
+  const float g = __fmul_rn(__uint_as_float((uint32_t)td.g[i] << 16), sg.gm);
+  float mn, vn;
+  moments(c, g, load1<MF>(td.m, i, sg.inv_s_m), load1<VF>(td.v, i, sg.inv_s_v), mn, vn);
+  am = fmax_nan(am, fabsf(mn));
+  av = fmax_nan(av, fabsf(vn));
+  uint32_t qm, qv;
+  const float mu = ext_q<MF, STATS, false>(a, mn, sg.s_m_new, sg.inv_s_m_new, rm, qm, flushed, sat);
+  const float vu = ext_q<VF, STATS, true>(a, vn, sg.s_v_new, sg.inv_s_v_new, rv, qv, flushed, sat);
+  if constexpr (MF == kFP32) static_cast<float*>(td.m)[i] = mn; else static_cast<uint8_t*>(td.m)[i] = (uint8_t)qm;
+  if constexpr (VF == kFP32) static_cast<float*>(td.v)[i] = vn; else static_cast<uint8_t*>(td.v)[i] = (uint8_t)qv;
+  const float pn = update(c, td.p[i], mu, vu);
+  td.p[i] = pn;
+  if (sg.pb) sg.pb[i] = __bfloat16_as_ushort(__float2bfloat16_rn(pn));
+}
+
+// 16 elements of an aligned tensor (vector loads/stores, as the default step).
+template <int MF, int VF, bool STATS>
+__device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& td, const ExtSeg& sg, int64_t i,
+                                            float& am, float& av, uint32_t& flushed, uint32_t& sat) {
+  const StepConsts& c = a.s.c;
+  float4 pv[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) pv[k] = ld_stream_f4(td.p + i + 4 * k);
+  const uint4 g0 = ld_ro_u4(td.g + i);
+  const uint4 g1 = ld_ro_u4(td.g + i + 8);
+  Tile16<MF> tm;
+  Tile16<VF> tv;
+  tm.load(td.m, i);
+  tv.load(td.v, i);
+  const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+  uint32_t pbw[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float mo[4], vo[4], mn[4], vn[4], mu[4], vu[4];
+    tm.decode4(k, sg.inv_s_m, mo);
+    tv.decode4(k, sg.inv_s_v, vo);
+    const float g[4] = {__fmul_rn(bf16_lo(gw[2 * k]), sg.gm), __fmul_rn(bf16_hi(gw[2 * k]), sg.gm),
+                        __fmul_rn(bf16_lo(gw[2 * k + 1]), sg.gm), __fmul_rn(bf16_hi(gw[2 * k + 1]), sg.gm)};
+    uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
+    if (a.flags & kExtStochastic) {
+      r0 = sr_words(a, sg.ti, (i + 4 * k) >> 1);
+      r1 = sr_words(a, sg.ti, ((i + 4 * k) >> 1) + 1);
+    }
+    const uint32_t rmj[4] = {r0.x, r0.z, r1.x, r1.z};
+    const uint32_t rvj[4] = {r0.y, r0.w, r1.y, r1.w};
+    uint32_t qm[4], qv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      moments(c, g[j], mo[j], vo[j], mn[j], vn[j]);
+      am = fmax_nan(am, fabsf(mn[j]));
+      av = fmax_nan(av, fabsf(vn[j]));
+      mu[j] = ext_q<MF, STATS, false>(a, mn[j], sg.s_m_new, sg.inv_s_m_new, rmj[j], qm[j], flushed, sat);
+      vu[j] = ext_q<VF, STATS, true>(a, vn[j], sg.s_v_new, sg.inv_s_v_new, rvj[j], qv[j], flushed, sat);
+    }
+    float pk[4] = {pv[k].x, pv[k].y, pv[k].z, pv[k].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) pk[j] = update(c, pk[j], mu[j], vu[j]);
+    pv[k] = make_float4(pk[0], pk[1], pk[2], pk[3]);
+    pbw[2 * k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(pk[0])) |
+                 ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(pk[1])) << 16);
+    pbw[2 * k + 1] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(pk[2])) |
+                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(pk[3])) << 16);
+    if constexpr (MF != kFP32) tm.w[k] = qm[0] | (qm[1] << 8) | (qm[2] << 16) | (qm[3] << 24);
+    else tm.r[k] = make_float4(mn[0], mn[1], mn[2], mn[3]);
+    if constexpr (VF != kFP32) tv.w[k] = qv[0] | (qv[1] << 8) | (qv[2] << 16) | (qv[3] << 24);
+    else tv.r[k] = make_float4(vn[0], vn[1], vn[2], vn[3]);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) st_stream_f4(td.p + i + 4 * k, pv[k]);
+  tm.store(td.m, i);
+  tv.store(td.v, i);
+  if (sg.pb) {  // 16 bf16 = 32 bytes; the bf16 buffer is 16-byte aligned when the tensor is
+    __stcs(reinterpret_cast<uint4*>(sg.pb + i), make_uint4(pbw[0], pbw[1], pbw[2], pbw[3]));
+    __stcs(reinterpret_cast<uint4*>(sg.pb + i + 8), make_uint4(pbw[4], pbw[5], pbw[6], pbw[7]));
+  }
+}
+
+// ------------------------------------------------------------ the variant step
+template <int MF, int VF, bool STATS>
+__device__ __forceinline__ void run_ext_segment(const ExtArgs& a, int ti, int64_t e0, int64_t e1, uint32_t units,
+                                                float gm, uint32_t (*red)[kThreads / 32]) {
+  const StepArgs& S = a.s;
+  const TensorDesc td = S.tensors[ti];
+  ExtSeg sg;
+  sg.ti = ti;
+  sg.gm = gm;
+  sg.pb = a.p_bf16 ? a.p_bf16[ti] : nullptr;
+  const float s_m = S.scale_m[ti], s_v = S.scale_v[ti];
+  float am_in = __uint_as_float(S.amax_in_m[ti]);
+  float av_in = __uint_as_float(S.amax_in_v[ti]);
+  if (a.use_hist) {
+    float hm = 0.0f, hv = 0.0f;
+    for (int k = 0; k < a.hist_len; ++k) {
+      hm = fmax_nan(hm, a.hist_m[(int64_t)k * S.num_tensors + ti]);
+      hv = fmax_nan(hv, a.hist_v[(int64_t)k * S.num_tensors + ti]);
+    }
+    am_in = hm;
+    av_in = hv;
+  }
+  sg.s_m_new = s_m;
+  sg.s_v_new = s_v;
+  if constexpr (MF != kFP32) sg.s_m_new = pow2scale_margin<MF>(am_in, s_m, a.margin_m);
+  if constexpr (VF != kFP32) sg.s_v_new = pow2scale_margin<VF>(av_in, s_v, a.margin_v);
+  sg.inv_s_m = __fdiv_rn(1.0f, s_m);
+  sg.inv_s_v = __fdiv_rn(1.0f, s_v);
+  sg.inv_s_m_new = __fdiv_rn(1.0f, sg.s_m_new);
+  sg.inv_s_v_new = __fdiv_rn(1.0f, sg.s_v_new);
+
+  float am = 0.0f, av = 0.0f;
+  uint32_t flushed = 0, sat = 0;
+  int64_t scalar_from = e0;
+  const bool vec = td.aligned && (sg.pb == nullptr || ((uintptr_t)sg.pb & 15u) == 0);
+  if (vec) {
+    for (int64_t i = e0 + (int64_t)threadIdx.x * kVec; i + kVec <= e1; i += kTile)
+      ext_group16<MF, VF, STATS>(a, td, sg, i, am, av, flushed, sat);
+    scalar_from = e0 + (e1 - e0) / kVec * kVec;
+  }
+  for (int64_t i = scalar_from + threadIdx.x; i < e1; i += kThreads)
+    ext_element<MF, VF, STATS>(a, td, sg, i, am, av, flushed, sat);
+
+  const uint32_t bm = block_max(__float_as_uint(am), red[0]);
+  const uint32_t bv = block_max(__float_as_uint(av), red[1]);
+  uint32_t bf = 0, bs = 0;
+  if constexpr (STATS) {
+    bf = block_sum(flushed, red[2]);
+    bs = block_sum(sat, red[3]);
+  }
+  if (threadIdx.x == 0) {
+    if (bm) atomicMax(S.acc_m + ti, bm);
+    if (bv) atomicMax(S.acc_v + ti, bv);
+    if constexpr (STATS) {
+      if (bf) atomicAdd(S.stats + 0, (unsigned long long)bf);
+      if (bs) atomicAdd(S.stats + 1, (unsigned long long)bs);
+    }
+    __threadfence();
+    const uint32_t prev = atomicAdd(S.done + ti, units);
+    if (prev + units == (uint32_t)td.nunits) {
+      __threadfence();
+      const uint32_t fm = atomicExch(S.acc_m + ti, 0u);
+      const uint32_t fv = atomicExch(S.acc_v + ti, 0u);
+      S.amax_m[ti] = __uint_as_float(fm);
+      S.amax_v[ti] = __uint_as_float(fv);
+      if (a.hist_m) {
+        a.hist_m[(int64_t)a.hist_slot * S.num_tensors + ti] = __uint_as_float(fm);
+        a.hist_v[(int64_t)a.hist_slot * S.num_tensors + ti] = __uint_as_float(fv);
+      }
+      S.scale_m[ti] = sg.s_m_new;
+      S.scale_v[ti] = sg.s_v_new;
+      S.done[ti] = 0u;
+    }
+  }
+}
+
+template <int MF, int VF, bool STATS>
+__global__ void __launch_bounds__(kThreads, 2)
+fp8adam_step_ext_kernel(const ExtArgs a) {
+  __shared__ uint32_t red[4][kThreads / 32];
+  if (a.skip && *a.skip) return;  // a non-finite gradient: the step is skipped
+  const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
+  for_each_segment(a.s, [&](int ti, int64_t e0, int64_t e1, uint32_t units) {
+    run_ext_segment<MF, VF, STATS>(a, ti, e0, e1, units, gm, red);
+  });
+}
+
+// ------------------------------------------------------------ amax pre-pass
+// Step-1 / current-scaling pre-pass of the variant step: the same moments
+// (with the gradient multiplier), no stores; accumulates into s.acc_m/acc_v.
+template <int MF, int VF>
+__global__ void __launch_bounds__(kThreads, 2)
+fp8adam_amax_ext_kernel(const ExtArgs a) {
+  __shared__ uint32_t red[2][kThreads / 32];
+  if (a.skip && *a.skip) return;
+  const StepArgs& S = a.s;
+  const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
+  for_each_segment(S, [&](int ti, int64_t e0, int64_t e1, uint32_t) {
+    const TensorDesc td = S.tensors[ti];
+    const float inv_s_m = __fdiv_rn(1.0f, S.scale_m[ti]);
+    const float inv_s_v = __fdiv_rn(1.0f, S.scale_v[ti]);
+    float am = 0.0f, av = 0.0f;
+    for (int64_t i = e0 + threadIdx.x; i < e1; i += kThreads) {
+      const float g = __fmul_rn(__uint_as_float((uint32_t)td.g[i] << 16), gm);
+      float mn, vn;
+      moments(S.c, g, load1<MF>(td.m, i, inv_s_m), load1<VF>(td.v, i, inv_s_v), mn, vn);
+      am = fmax_nan(am, fabsf(mn));
+      av = fmax_nan(av, fabsf(vn));
+    }
+    const uint32_t bm = block_max(__float_as_uint(am), red[0]);
+    const uint32_t bv = block_max(__float_as_uint(av), red[1]);
+    if (threadIdx.x == 0) {
+      if (bm) atomicMax(S.acc_m + ti, bm);
+      if (bv) atomicMax(S.acc_v + ti, bv);
+    }
+  });
+}
+
+// ------------------------------------------------------------ grad-norm pre-pass
+// Per CTA: the sum of g^2 (each term exact in double) over its tiles, in a
+// fixed order (thread-sequential, then a fixed shuffle/shared-memory tree),
+// written to partial[blockIdx.x]; non-finite gradients are counted (not
+// summed).  The fixed grid makes the result reproducible run to run.
+__device__ __forceinline__ double block_sum_d(double x, double* sm) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) sm[warp] = x;
+  __syncthreads();
+  double r = 0.0;
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) r += sm[w];
+  }
+  return r;
+}
+
+__global__ void __launch_bounds__(kThreads)
+fp8adam_gradnorm_partial_kernel(const StepArgs a, double* partial, unsigned long long* nonfinite) {
+  __shared__ double red[kThreads / 32];
+  __shared__ uint32_t redi[kThreads / 32];
+  double acc = 0.0;
+  uint32_t bad = 0;
+  for_each_segment(a, [&](int ti, int64_t e0, int64_t e1, uint32_t) {
+    const uint16_t* g = a.tensors[ti].g;
+    for (int64_t i = e0 + threadIdx.x; i < e1; i += kThreads) {
+      const uint32_t b = g[i];
+      if ((b & 0x7F80u) == 0x7F80u) {
+        ++bad;
+      } else {
+        const double x = (double)__uint_as_float(b << 16);
+        acc = __dadd_rn(acc, __dmul_rn(x, x));
+      }
+    }
+  });
+  const double s = block_sum_d(acc, red);
+  const uint32_t nb = block_sum(bad, redi);
+  if (threadIdx.x == 0) {
+    partial[blockIdx.x] = s;
+    if (nb) atomicAdd(nonfinite, (unsigned long long)nb);
+  }
+}
+
+// One CTA: the fixed-order total, the multiplier and the skip flag.
+// c = (1/loss_scale) * min(1, max_norm / (norm + 1e-6)), norm = sqrt(sum)/loss_scale
+// (clip_grad_norm_'s definition on the unscaled gradients); max_norm <= 0 =
+// no clipping; all in double, c rounded once to fp32.
+__global__ void __launch_bounds__(kThreads)
+fp8adam_gradnorm_finalize_kernel(const double* partial, int n, const unsigned long long* nonfinite,
+                                 float loss_scale, float max_norm, int skip_nonfinite, float* grad_mult,
+                                 uint32_t* skip, double* norm_out) {
+  __shared__ double red[kThreads / 32];
+  double acc = 0.0;
+  for (int k = threadIdx.x; k < n; k += kThreads) acc = __dadd_rn(acc, partial[k]);
+  const double sum = block_sum_d(acc, red);
+  if (threadIdx.x == 0) {
+    const double inv = __ddiv_rn(1.0, (double)loss_scale);
+    const double norm = __dmul_rn(__dsqrt_rn(sum), inv);
+    double coef = 1.0;
+    if (max_norm > 0.0f) {
+      coef = __ddiv_rn((double)max_norm, __dadd_rn(norm, 1e-6));
+      if (coef > 1.0) coef = 1.0;
+    }
+    *grad_mult = __double2float_rn(__dmul_rn(inv, coef));
+    *norm_out = norm;
+    *skip = (skip_nonfinite && *nonfinite != 0ull) ? 1u : 0u;
+  }
+}
+
+}  // namespace fp8adam

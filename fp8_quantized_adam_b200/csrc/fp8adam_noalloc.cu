@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kThreads) noalloc_kernel(const NoAllocArgs a) 
     if constexpr (WRITE) {
       __threadfence();
       const uint32_t prev = atomicAdd(a.done + ti, 1u);
-      if (prev == (uint32_t)td.nchunks - 1u) {
+      if (prev == (uint32_t)td.nunits - 1u) {
         __threadfence();
         a.amax_m[ti] = __uint_as_float(atomicExch(a.acc_m + ti, 0u));
         a.amax_v[ti] = __uint_as_float(atomicExch(a.acc_v + ti, 0u));
@@ -240,7 +240,7 @@ extern "C" int fp8adam_step_noalloc(const fp8adam_tensor* tensors, int32_t num_t
     d.numel = t.numel;
     const int64_t nc = (t.numel + kChunk - 1) / kChunk;
     if (nc > INT32_MAX) return FP8ADAM_ERR_INVALID_ARG;
-    d.nchunks = (int32_t)nc;
+    d.nunits = (int32_t)nc;
     d.aligned = aligned16(t.param) && aligned16(t.grad) && aligned16(t.m) && aligned16(t.v);
     g_host_image.begin[i] = (int32_t)chunks;
     chunks += nc;

@@ -9,14 +9,16 @@
 //
 // Design for B200: the step is a pure HBM stream (read p 4 B, g 2 B, m 1 B,
 // v 1 B; write p 4 B, m 1 B, v 1 B per element).  One launch covers a whole
-// parameter list through a chunk table: CTA b handles chunk b, a range of at
-// most kChunk elements of one tensor.  Each thread moves 16 elements per
-// iteration with 16-byte loads and stores (4 x p, 2 x g, 1 x m, 1 x v),
-// streaming cache hints, all fp32 arithmetic as single IEEE operations (no
-// FMA contraction), hardware cvt for the FP8 conversions.  The new amax of a
-// tensor is reduced with a warp redux and one atomicMax per CTA; the CTA that
-// completes a tensor's last chunk (per-tensor counter) publishes its amax and
-// scale, so a step is a single kernel (plus an amax pre-pass at step 1).
+// parameter list.  The list is cut into tiles of kTile elements (a tensor's
+// last tile may be short); a persistent grid of (SMs x resident CTAs) CTAs
+// takes contiguous, equal ranges of the global tile sequence.  Within a tile
+// each thread moves 16 elements with 16-byte loads and stores (4 x p, 2 x g,
+// 1 x m, 1 x v), streaming cache hints, all fp32 arithmetic as single IEEE
+// operations (no FMA contraction), hardware cvt for the FP8 conversions.  A
+// CTA keeps the running amax of the tensor it is in, and flushes it once per
+// tensor segment (warp redux, one atomicMax per moment); the CTA whose flush
+// completes a tensor's tile count publishes its amax and scale, so a step is
+// a single kernel (plus an amax pre-pass at step 1).
 #pragma once
 
 #include <stdint.h>
@@ -26,9 +28,16 @@
 namespace fp8adam {
 
 constexpr int kThreads = 256;
-constexpr int kVec = 16;                     // elements per thread per iteration
-constexpr int kTile = kThreads * kVec;       // 4096 elements per CTA iteration
-constexpr int64_t kChunk = 16 * (int64_t)kTile;  // 65536 elements per CTA
+constexpr int kVec = 16;                     // elements per thread per tile
+constexpr int kTile = kThreads * kVec;       // 4096 elements per tile
+constexpr int64_t kChunk = 16 * (int64_t)kTile;  // 65536: work unit of the allocation-free path
+
+// resident CTAs per SM the step kernel is built for (register budget): FP8
+// moments fit 64 registers per thread (4 x 256 threads), fp32 moments 128
+template <int MF, int VF>
+struct StepOccupancy {
+  static constexpr int kMinBlocks = (MF != 2 && VF != 2) ? 4 : 2;
+};
 
 struct TensorDesc {
   float* p;
@@ -36,13 +45,15 @@ struct TensorDesc {
   void* m;
   void* v;
   int64_t numel;
-  int32_t nchunks;
+  int32_t nunits;   // work units of the tensor (tiles of the step kernel, chunks
+                    // of the allocation-free path)
   int32_t aligned;  // all four buffers 16-byte aligned
 };
 
+// One chunk of the chunk schedule: kChunk elements of a tensor from `start`.
 struct Chunk {
   int32_t tensor;
-  int32_t len;
+  int32_t pad;
   int64_t start;
 };
 
@@ -51,8 +62,12 @@ struct StepConsts {
 };
 
 struct StepArgs {
-  const TensorDesc* tensors;
-  const Chunk* chunks;
+  const TensorDesc* tensors;     // [T]
+  const int32_t* unit_begin;     // [T+1] first work unit (chunk or tile) of each tensor
+  const Chunk* chunks;           // chunk schedule: [total units] tensor and start of each chunk
+  int32_t num_tensors;
+  int32_t total_tiles;           // persistent schedule: tiles of the whole list
+  int32_t tiles_per_cta;         // persistent schedule: contiguous range of each CTA
   float* scale_m;            // [T] in: decode scale; out: encode scale of this step
   float* scale_v;
   float* amax_m;             // [T] out: max |m| of this step
@@ -61,7 +76,7 @@ struct StepArgs {
   const uint32_t* amax_in_v;
   uint32_t* acc_m;           // [T] amax accumulators (bits), zero between steps
   uint32_t* acc_v;
-  uint32_t* done;            // [T] finished-chunk counters, zero between steps
+  uint32_t* done;            // [T] finished-tile counters, zero between steps
   unsigned long long* stats; // [2] flushed, saturated (STATS only)
   StepConsts c;
 };
@@ -116,6 +131,21 @@ __device__ __forceinline__ float update(const StepConsts& c, float p, float m, f
 }
 
 __device__ __forceinline__ uint32_t umax(uint32_t a, uint32_t b) { return a > b ? a : b; }
+// max that returns NaN if either input is NaN (the canonical, positive NaN)
+#ifndef FP8ADAM_AMAX_INT
+#define FP8ADAM_AMAX_INT 0
+#endif
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+#if FP8ADAM_AMAX_INT
+  // both non-negative or NaN: integer max of the bits keeps NaN (its bits
+  // exceed those of inf)
+  return __uint_as_float(umax(__float_as_uint(a), __float_as_uint(b) & 0x7FFFFFFFu));
+#else
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+#endif
+}
 // |x| as ordered bits: integer max over them is a float max that keeps NaN
 __device__ __forceinline__ uint32_t abs_bits(float x) { return __float_as_uint(x) & 0x7FFFFFFFu; }
 
@@ -230,167 +260,191 @@ __device__ __forceinline__ uint32_t block_sum(uint32_t x, uint32_t* sm) {
   return r;
 }
 
-// ------------------------------------------------------------ step kernel
-template <int MF, int VF, bool STATS>
-__global__ void __launch_bounds__(kThreads)
-fp8adam_step_kernel(const StepArgs a) {
-  __shared__ uint32_t red[4][kThreads / 32];
-  const Chunk ch = a.chunks[blockIdx.x];
-  const int ti = ch.tensor;
-  const TensorDesc td = a.tensors[ti];
-  const StepConsts c = a.c;
-
-  const float s_m = a.scale_m[ti];
-  const float s_v = a.scale_v[ti];
-  float s_m_new = s_m, s_v_new = s_v;
-  if constexpr (MF != kFP32) s_m_new = pow2scale<MF>(__uint_as_float(a.amax_in_m[ti]), s_m);
-  if constexpr (VF != kFP32) s_v_new = pow2scale<VF>(__uint_as_float(a.amax_in_v[ti]), s_v);
-  const float inv_s_m = __fdiv_rn(1.0f, s_m);  // exact: powers of two
-  const float inv_s_v = __fdiv_rn(1.0f, s_v);
-
-  uint32_t am = 0, av = 0, flushed = 0, sat = 0;
-  const int64_t start = ch.start;
-  const int64_t end = ch.start + ch.len;
-  int64_t scalar_from = start;
-
-  if (td.aligned) {
-    const int64_t vec_end = start + (int64_t)(ch.len / kVec) * kVec;
-    for (int64_t i = start + (int64_t)threadIdx.x * kVec; i < vec_end; i += kTile) {
-      float4 pv[4];
+// ------------------------------------------------------------ tile bodies
+// One full 16-element group per thread of an aligned tensor (vector path).
+template <int MF, int VF, bool STATS, bool WRITE>
+__device__ __forceinline__ void group16(const TensorDesc& td, int64_t i, const StepConsts& c, float inv_s_m,
+                                        float inv_s_v, float s_m_new, float s_v_new, float& am, float& av,
+                                        uint32_t& flushed, uint32_t& sat) {
+  float4 pv[4];
+  if constexpr (WRITE) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) pv[k] = ld_stream_f4(td.p + i + 4 * k);
-      const uint4 g0 = ld_ro_u4(td.g + i);
-      const uint4 g1 = ld_ro_u4(td.g + i + 8);
-      Tile16<MF> tm;
-      Tile16<VF> tv;
-      tm.load(td.m, i);
-      tv.load(td.v, i);
-      const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float mo[4], vo[4], mn[4], vn[4];
-        tm.decode4(k, inv_s_m, mo);
-        tv.decode4(k, inv_s_v, vo);
-        const float g[4] = {bf16_lo(gw[2 * k]), bf16_hi(gw[2 * k]), bf16_lo(gw[2 * k + 1]),
-                            bf16_hi(gw[2 * k + 1])};
-        float pk[4] = {pv[k].x, pv[k].y, pv[k].z, pv[k].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          moments(c, g[j], mo[j], vo[j], mn[j], vn[j]);
-          am = umax(am, abs_bits(mn[j]));
-          av = umax(av, abs_bits(vn[j]));
-          pk[j] = update(c, pk[j], mn[j], vn[j]);
-        }
-        pv[k] = make_float4(pk[0], pk[1], pk[2], pk[3]);
-        tm.template encode4<STATS, false>(k, s_m_new, mn, flushed, sat);
-        tv.template encode4<STATS, true>(k, s_v_new, vn, flushed, sat);
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) st_stream_f4(td.p + i + 4 * k, pv[k]);
-      tm.store(td.m, i);
-      tv.store(td.v, i);
-    }
-    scalar_from = vec_end;
+    for (int k = 0; k < 4; ++k) pv[k] = ld_stream_f4(td.p + i + 4 * k);
   }
-  for (int64_t i = scalar_from + threadIdx.x; i < end; i += kThreads) {
-    const float g = __uint_as_float((uint32_t)td.g[i] << 16);
-    const float mo = load1<MF>(td.m, i, inv_s_m);
-    const float vo = load1<VF>(td.v, i, inv_s_v);
-    float mn, vn;
-    moments(c, g, mo, vo, mn, vn);
-    am = umax(am, abs_bits(mn));
-    av = umax(av, abs_bits(vn));
+  const uint4 g0 = ld_ro_u4(td.g + i);
+  const uint4 g1 = ld_ro_u4(td.g + i + 8);
+  Tile16<MF> tm;
+  Tile16<VF> tv;
+  tm.load(td.m, i);
+  tv.load(td.v, i);
+  const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float mo[4], vo[4], mn[4], vn[4];
+    tm.decode4(k, inv_s_m, mo);
+    tv.decode4(k, inv_s_v, vo);
+    const float g[4] = {bf16_lo(gw[2 * k]), bf16_hi(gw[2 * k]), bf16_lo(gw[2 * k + 1]), bf16_hi(gw[2 * k + 1])};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      moments(c, g[j], mo[j], vo[j], mn[j], vn[j]);
+      am = fmax_nan(am, fabsf(mn[j]));
+      av = fmax_nan(av, fabsf(vn[j]));
+    }
+    if constexpr (WRITE) {
+      float pk[4] = {pv[k].x, pv[k].y, pv[k].z, pv[k].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) pk[j] = update(c, pk[j], mn[j], vn[j]);
+      pv[k] = make_float4(pk[0], pk[1], pk[2], pk[3]);
+      tm.template encode4<STATS, false>(k, s_m_new, mn, flushed, sat);
+      tv.template encode4<STATS, true>(k, s_v_new, vn, flushed, sat);
+    }
+  }
+  if constexpr (WRITE) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) st_stream_f4(td.p + i + 4 * k, pv[k]);
+    tm.store(td.m, i);
+    tv.store(td.v, i);
+  }
+}
+
+// One element (ragged tails, unaligned tensors).
+template <int MF, int VF, bool STATS, bool WRITE>
+__device__ __forceinline__ void element1(const TensorDesc& td, int64_t i, const StepConsts& c, float inv_s_m,
+                                         float inv_s_v, float s_m_new, float s_v_new, float& am, float& av,
+                                         uint32_t& flushed, uint32_t& sat) {
+  const float g = __uint_as_float((uint32_t)td.g[i] << 16);
+  float mn, vn;
+  moments(c, g, load1<MF>(td.m, i, inv_s_m), load1<VF>(td.v, i, inv_s_v), mn, vn);
+  am = fmax_nan(am, fabsf(mn));
+  av = fmax_nan(av, fabsf(vn));
+  if constexpr (WRITE) {
     td.p[i] = update(c, td.p[i], mn, vn);
     store1<MF, STATS, false>(td.m, i, mn, s_m_new, flushed, sat);
     store1<VF, STATS, true>(td.v, i, vn, s_v_new, flushed, sat);
   }
+}
 
-  const uint32_t bm = block_max(am, red[0]);
-  const uint32_t bv = block_max(av, red[1]);
+// ------------------------------------------------------------ one segment
+// The element range [e0, e1) of tensor ti: moments, update, codes, then the
+// amax flush.  `units` is the number of work units the range stands for;
+// the flush that brings the tensor's count to td.nunits publishes its amax
+// and scale (every CTA that reads them for this step has done so by then).
+// WRITE = false is the amax pre-pass (no stores, nothing published).
+template <int MF, int VF, bool STATS, bool WRITE>
+__device__ __forceinline__ void run_segment(const StepArgs& a, int ti, int64_t e0, int64_t e1, uint32_t units,
+                                            uint32_t (*red)[kThreads / 32]) {
+  const TensorDesc td = a.tensors[ti];
+  const StepConsts c = a.c;
+  const float s_m = a.scale_m[ti];
+  const float s_v = a.scale_v[ti];
+  float s_m_new = s_m, s_v_new = s_v;
+  if constexpr (WRITE && MF != kFP32) s_m_new = pow2scale<MF>(__uint_as_float(a.amax_in_m[ti]), s_m);
+  if constexpr (WRITE && VF != kFP32) s_v_new = pow2scale<VF>(__uint_as_float(a.amax_in_v[ti]), s_v);
+  const float inv_s_m = __fdiv_rn(1.0f, s_m);  // exact: powers of two
+  const float inv_s_v = __fdiv_rn(1.0f, s_v);
+
+  float am = 0.0f, av = 0.0f;
+  uint32_t flushed = 0, sat = 0;
+  int64_t scalar_from = e0;
+  if (td.aligned) {
+    for (int64_t i = e0 + (int64_t)threadIdx.x * kVec; i + kVec <= e1; i += kTile)
+      group16<MF, VF, STATS, WRITE>(td, i, c, inv_s_m, inv_s_v, s_m_new, s_v_new, am, av, flushed, sat);
+    scalar_from = e0 + (e1 - e0) / kVec * kVec;
+  }
+  for (int64_t i = scalar_from + threadIdx.x; i < e1; i += kThreads)
+    element1<MF, VF, STATS, WRITE>(td, i, c, inv_s_m, inv_s_v, s_m_new, s_v_new, am, av, flushed, sat);
+
+  const uint32_t bm = block_max(__float_as_uint(am), red[0]);
+  const uint32_t bv = block_max(__float_as_uint(av), red[1]);
   uint32_t bf = 0, bs = 0;
-  if constexpr (STATS) {
+  if constexpr (STATS && WRITE) {
     bf = block_sum(flushed, red[2]);
     bs = block_sum(sat, red[3]);
   }
   if (threadIdx.x == 0) {
     if (bm) atomicMax(a.acc_m + ti, bm);
     if (bv) atomicMax(a.acc_v + ti, bv);
-    if constexpr (STATS) {
-      if (bf) atomicAdd(a.stats + 0, (unsigned long long)bf);
-      if (bs) atomicAdd(a.stats + 1, (unsigned long long)bs);
-    }
-    // the CTA finishing a tensor's last chunk publishes its amax and scale;
-    // every other CTA of the tensor has finished reading them by then
-    __threadfence();
-    const uint32_t prev = atomicAdd(a.done + ti, 1u);
-    if (prev == (uint32_t)td.nchunks - 1u) {
+    if constexpr (WRITE) {
+      if constexpr (STATS) {
+        if (bf) atomicAdd(a.stats + 0, (unsigned long long)bf);
+        if (bs) atomicAdd(a.stats + 1, (unsigned long long)bs);
+      }
       __threadfence();
-      a.amax_m[ti] = __uint_as_float(atomicExch(a.acc_m + ti, 0u));
-      a.amax_v[ti] = __uint_as_float(atomicExch(a.acc_v + ti, 0u));
-      a.scale_m[ti] = s_m_new;
-      a.scale_v[ti] = s_v_new;
-      a.done[ti] = 0u;
+      const uint32_t prev = atomicAdd(a.done + ti, units);
+      if (prev + units == (uint32_t)td.nunits) {
+        __threadfence();
+        a.amax_m[ti] = __uint_as_float(atomicExch(a.acc_m + ti, 0u));
+        a.amax_v[ti] = __uint_as_float(atomicExch(a.acc_v + ti, 0u));
+        a.scale_m[ti] = s_m_new;
+        a.scale_v[ti] = s_v_new;
+        a.done[ti] = 0u;
+      }
     }
   }
 }
 
-// ------------------------------------------------------------ amax pre-pass
-// Same moments as the step, no stores: this step's own amax (step 1, or
-// every step in "current" scaling), accumulated into acc_m/acc_v.
+// ------------------------------------------------------------ the schedule
+// How a launch's CTAs cover the parameter list.  f(ti, e0, e1, units) is
+// called for each segment (an element range [e0, e1) of tensor ti standing
+// for `units` work units) of this CTA, in order.
+#ifndef FP8ADAM_PERSISTENT
+#define FP8ADAM_PERSISTENT 0
+#endif
+#if FP8ADAM_PERSISTENT
+// persistent grid: CTA b takes the contiguous tile range [b*tiles_per_cta,
+// (b+1)*tiles_per_cta) of the whole list; work units are tiles (kTile)
+constexpr int64_t kUnit = kTile;
+template <typename F>
+__device__ __forceinline__ void for_each_segment(const StepArgs& a, F&& f) {
+  const int32_t g0 = (int32_t)blockIdx.x * a.tiles_per_cta;
+  const int32_t g1 = min(g0 + a.tiles_per_cta, a.total_tiles);
+  if (g0 >= g1) return;
+  int lo = 0, hi = a.num_tensors;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (a.unit_begin[mid] <= g0) lo = mid; else hi = mid;
+  }
+  int ti = lo;
+  int32_t gt = g0;
+  while (gt < g1) {
+    while (a.unit_begin[ti + 1] <= gt) ++ti;  // skip empty tensors
+    const int32_t tb = a.unit_begin[ti];
+    const int32_t seg_end = min(a.unit_begin[ti + 1], g1);
+    f(ti, (int64_t)(gt - tb) * kTile, min((int64_t)(seg_end - tb) * kTile, a.tensors[ti].numel),
+      (uint32_t)(seg_end - gt));
+    __syncthreads();  // shared reduction buffers are reused by the next segment
+    gt = seg_end;
+    ++ti;
+  }
+}
+#else
+// one CTA per chunk: work units are chunks of kChunk elements of one tensor
+constexpr int64_t kUnit = kChunk;
+template <typename F>
+__device__ __forceinline__ void for_each_segment(const StepArgs& a, F&& f) {
+  const Chunk ch = a.chunks[blockIdx.x];  // one 16-byte load: the tensor and the start
+  f(ch.tensor, ch.start, min(ch.start + kChunk, a.tensors[ch.tensor].numel), 1u);
+}
+#endif
+
+template <int MF, int VF, bool STATS, bool WRITE>
+__device__ __forceinline__ void step_body(const StepArgs& a) {
+  __shared__ uint32_t red[4][kThreads / 32];
+  for_each_segment(a, [&](int ti, int64_t e0, int64_t e1, uint32_t units) {
+    run_segment<MF, VF, STATS, WRITE>(a, ti, e0, e1, units, red);
+  });
+}
+
+template <int MF, int VF, bool STATS>
+__global__ void __launch_bounds__(kThreads, StepOccupancy<MF, VF>::kMinBlocks)
+fp8adam_step_kernel(const StepArgs a) {
+  step_body<MF, VF, STATS, true>(a);
+}
+
 template <int MF, int VF>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, StepOccupancy<MF, VF>::kMinBlocks)
 fp8adam_amax_kernel(const StepArgs a) {
-  __shared__ uint32_t red[2][kThreads / 32];
-  const Chunk ch = a.chunks[blockIdx.x];
-  const int ti = ch.tensor;
-  const TensorDesc td = a.tensors[ti];
-  const StepConsts c = a.c;
-  const float inv_s_m = __fdiv_rn(1.0f, a.scale_m[ti]);
-  const float inv_s_v = __fdiv_rn(1.0f, a.scale_v[ti]);
-  uint32_t am = 0, av = 0;
-  const int64_t start = ch.start, end = ch.start + ch.len;
-  int64_t scalar_from = start;
-  if (td.aligned) {
-    const int64_t vec_end = start + (int64_t)(ch.len / kVec) * kVec;
-    for (int64_t i = start + (int64_t)threadIdx.x * kVec; i < vec_end; i += kTile) {
-      const uint4 g0 = ld_ro_u4(td.g + i);
-      const uint4 g1 = ld_ro_u4(td.g + i + 8);
-      Tile16<MF> tm;
-      Tile16<VF> tv;
-      tm.load(td.m, i);
-      tv.load(td.v, i);
-      const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float mo[4], vo[4];
-        tm.decode4(k, inv_s_m, mo);
-        tv.decode4(k, inv_s_v, vo);
-        const float g[4] = {bf16_lo(gw[2 * k]), bf16_hi(gw[2 * k]), bf16_lo(gw[2 * k + 1]),
-                            bf16_hi(gw[2 * k + 1])};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float mn, vn;
-          moments(c, g[j], mo[j], vo[j], mn, vn);
-          am = umax(am, abs_bits(mn));
-          av = umax(av, abs_bits(vn));
-        }
-      }
-    }
-    scalar_from = vec_end;
-  }
-  for (int64_t i = scalar_from + threadIdx.x; i < end; i += kThreads) {
-    const float g = __uint_as_float((uint32_t)td.g[i] << 16);
-    float mn, vn;
-    moments(c, g, load1<MF>(td.m, i, inv_s_m), load1<VF>(td.v, i, inv_s_v), mn, vn);
-    am = umax(am, abs_bits(mn));
-    av = umax(av, abs_bits(vn));
-  }
-  const uint32_t bm = block_max(am, red[0]);
-  const uint32_t bv = block_max(av, red[1]);
-  if (threadIdx.x == 0) {
-    if (bm) atomicMax(a.acc_m + ti, bm);
-    if (bv) atomicMax(a.acc_v + ti, bv);
-  }
+  step_body<MF, VF, false, false>(a);
 }
 
 }  // namespace fp8adam

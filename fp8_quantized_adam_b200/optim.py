@@ -8,6 +8,7 @@ bit for bit.
 """
 from __future__ import annotations
 
+import ctypes
 from typing import List, Optional, Sequence
 
 import torch
@@ -28,6 +29,13 @@ class FP8AdamW:
     allocated (zeros) unless given; ``m_fmt``/``v_fmt`` default to E4M3/E5M2.
     The tensors must keep their storage (addresses) for the optimizer's
     lifetime.
+
+    Options (fp8adam_create_ex): ``margin_m``/``margin_v`` (scale margin),
+    ``amax_history_len`` (scale from the max of the last N amax; the ring is
+    allocated here and checkpointed), ``update_from_stored`` (the update reads
+    the requantised moments), ``stochastic_rounding`` with ``seed``, and
+    ``param_bf16`` (bf16 tensors receiving the updated params).  Per step:
+    ``step(loss_scale=, max_norm=, skip_nonfinite=)`` (fp8adam_step_ex).
     """
 
     def __init__(self, params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor], *,
@@ -36,7 +44,10 @@ class FP8AdamW:
                  v: Optional[List[torch.Tensor]] = None, scale_m: Optional[torch.Tensor] = None,
                  scale_v: Optional[torch.Tensor] = None, amax_m: Optional[torch.Tensor] = None,
                  amax_v: Optional[torch.Tensor] = None, stats: bool = False,
-                 jit_every_step: bool = False):
+                 jit_every_step: bool = False, margin_m: int = 0, margin_v: int = 0,
+                 amax_history_len: int = 0, update_from_stored: bool = False,
+                 stochastic_rounding: bool = False, seed: int = 0,
+                 param_bf16: Optional[List[torch.Tensor]] = None):
         if len(params) == 0 or len(params) != len(grads):
             raise ValueError("need matching, non-empty param and grad lists")
         self.params, self.grads = list(params), list(grads)
@@ -68,20 +79,52 @@ class FP8AdamW:
         arr = (capi.fp8adam_tensor * T)()
         for i, (p, g, mm, vv) in enumerate(zip(self.params, self.grads, self.m, self.v)):
             arr[i] = capi.fp8adam_tensor(p.data_ptr(), g.data_ptr(), mm.data_ptr(), vv.data_ptr(), p.numel())
-        flags = (capi.FLAG_STATS if stats else 0) | (capi.FLAG_JIT_EVERY_STEP if jit_every_step else 0)
+        flags = ((capi.FLAG_STATS if stats else 0) | (capi.FLAG_JIT_EVERY_STEP if jit_every_step else 0)
+                 | (capi.FLAG_UPDATE_FROM_STORED if update_from_stored else 0)
+                 | (capi.FLAG_STOCHASTIC_ROUNDING if stochastic_rounding else 0))
+        self.amax_history_len = int(amax_history_len)
+        self.hist_m = self.hist_v = None
+        if self.amax_history_len > 1:
+            self.hist_m = torch.zeros(self.amax_history_len, T, dtype=torch.float32, device=dev)
+            self.hist_v = torch.zeros(self.amax_history_len, T, dtype=torch.float32, device=dev)
+        self.param_bf16 = list(param_bf16) if param_bf16 is not None else None
+        bf16_arr = None
+        if self.param_bf16 is not None:
+            if len(self.param_bf16) != T:
+                raise ValueError("need one bf16 output per param")
+            bf16_arr = (ctypes.c_void_p * T)(*[b.data_ptr() for b in self.param_bf16])
+        opts = capi.fp8adam_options(self.scale_m.data_ptr(), self.scale_v.data_ptr(), self.amax_m.data_ptr(),
+                                    self.amax_v.data_ptr(), self.m_fmt, self.v_fmt, flags, margin_m, margin_v,
+                                    self.amax_history_len,
+                                    self.hist_m.data_ptr() if self.hist_m is not None else None,
+                                    self.hist_v.data_ptr() if self.hist_v is not None else None,
+                                    seed, ctypes.cast(bf16_arr, ctypes.c_void_p) if bf16_arr is not None else None)
         with torch.cuda.device(dev):
-            self.ctx = capi.fp8adam_create(arr, T, self.scale_m.data_ptr(), self.scale_v.data_ptr(),
-                                           self.amax_m.data_ptr(), self.amax_v.data_ptr(),
-                                           self.m_fmt, self.v_fmt, flags)
+            self.ctx = capi.fp8adam_create_ex(arr, T, opts)
         self.device = dev
 
-    def step(self, stream: Optional[torch.cuda.Stream] = None, lr: Optional[float] = None) -> None:
+    def step(self, stream: Optional[torch.cuda.Stream] = None, lr: Optional[float] = None,
+             loss_scale: float = 1.0, max_norm: float = 0.0, skip_nonfinite: bool = False) -> None:
         """One AdamW step on every tensor, queued on ``stream`` (default: the
-        current torch stream).  Never synchronises."""
+        current torch stream).  Never synchronises.  ``loss_scale`` divides
+        the gradients, ``max_norm`` > 0 clips their global L2 norm,
+        ``skip_nonfinite`` skips the whole step on an inf/NaN gradient."""
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         self.t += 1
-        capi.fp8adam_step(self.ctx, self.lr if lr is None else lr, self.betas[0], self.betas[1], self.eps,
-                          self.weight_decay, self.t, s.cuda_stream)
+        lr = self.lr if lr is None else lr
+        if loss_scale == 1.0 and max_norm <= 0.0 and not skip_nonfinite:
+            capi.fp8adam_step(self.ctx, lr, self.betas[0], self.betas[1], self.eps, self.weight_decay, self.t,
+                              s.cuda_stream)
+        else:
+            sp = capi.fp8adam_step_params(lr, self.betas[0], self.betas[1], self.eps, self.weight_decay, self.t,
+                                          loss_scale, max_norm, 1 if skip_nonfinite else 0)
+            capi.fp8adam_step_ex(self.ctx, sp, s.cuda_stream)
+
+    def grad_info(self, stream: Optional[torch.cuda.Stream] = None):
+        """(global grad L2 norm, skipped) of the last step with a gradient
+        pre-pass (synchronises the stream)."""
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        return capi.fp8adam_get_grad_info(self.ctx, s.cuda_stream)
 
     def stats(self, stream: Optional[torch.cuda.Stream] = None):
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
@@ -97,7 +140,9 @@ class FP8AdamW:
                 "m": [x.clone() for x in self.m], "v": [x.clone() for x in self.v],
                 "scale_m": self.scale_m.clone(), "scale_v": self.scale_v.clone(),
                 "amax_m": self.amax_m.clone(), "amax_v": self.amax_v.clone(),
-                "m_fmt": self.m_fmt, "v_fmt": self.v_fmt}
+                "m_fmt": self.m_fmt, "v_fmt": self.v_fmt,
+                "amax_history_m": None if self.hist_m is None else self.hist_m.clone(),
+                "amax_history_v": None if self.hist_v is None else self.hist_v.clone()}
 
     def load_state_dict(self, sd: dict) -> None:
         if sd["m_fmt"] != self.m_fmt or sd["v_fmt"] != self.v_fmt:
@@ -111,6 +156,9 @@ class FP8AdamW:
                 dst.copy_(src)
             for name in ("scale_m", "scale_v", "amax_m", "amax_v"):
                 getattr(self, name).copy_(sd[name])
+            if self.hist_m is not None:
+                self.hist_m.copy_(sd["amax_history_m"])
+                self.hist_v.copy_(sd["amax_history_v"])
         self.t = int(sd["t"])
 
     def close(self) -> None:

@@ -130,6 +130,75 @@ int fp8adam_destroy(fp8adam_ctx* ctx);
 /* Static description of an error code. */
 const char* fp8adam_strerror(int code);
 
+/* ---- options: scaling and read-back variants, stochastic rounding, fused
+ * loss-scale removal / clipping / skip-on-non-finite, bf16 param copy -----
+ * Sources: "FP8训练的稳定性挑战…", section "应对FP8训练稳定性挑战的策略"
+ * (stochastic rounding, gradient clipping, adaptive gradient scaling), its
+ * GradScaler / clip_grad_norm_ examples and the transformer_engine
+ * DelayedScaling example (margin, amax_history_len, amax algo MAX); the
+ * daoxuan.cc explainer's numeric example (v cut to 0 -> 1/(0+eps)) for the
+ * update from stored moments. */
+#define FP8ADAM_FLAG_UPDATE_FROM_STORED 4u   /* the update reads dec(code)/scale */
+#define FP8ADAM_FLAG_STOCHASTIC_ROUNDING 8u  /* codes rounded stochastically */
+
+typedef struct {
+  float* scale_m;            /* as fp8adam_create: device fp32 [num_tensors] */
+  float* scale_v;
+  float* amax_m;
+  float* amax_v;
+  int32_t m_fmt;             /* fp8adam_fmt */
+  int32_t v_fmt;
+  uint32_t flags;            /* FP8ADAM_FLAG_* */
+  int32_t margin_m;          /* scale = 2^(k - margin), k as above; 0..64 */
+  int32_t margin_v;
+  int32_t amax_history_len;  /* <= 1: the previous step's amax; > 1 (<= 1024): the
+                                max over the last amax_history_len steps */
+  float* amax_history_m;     /* device fp32 [amax_history_len][num_tensors], zero
+                                at the start of training, caller-owned (part of the
+                                checkpointed state); slot (step-1) % len holds the
+                                amax of that step.  NULL when len <= 1. */
+  float* amax_history_v;
+  uint64_t seed;             /* stochastic rounding: random bits of element j of
+                                tensor i at step t for moment w (0 = m, 1 = v) are
+                                word 2*(j&1) + w of Philox4x32-10 with counter
+                                (j/2 low, j/2 high, i, t low 32 bits) and key
+                                (seed low, seed high); a code rounds up to the
+                                next grid value iff r*(hi-lo) < (|x|-lo)*2^32 */
+  uint16_t* const* param_bf16; /* host array [num_tensors] of device bf16 buffers
+                                  [numel] receiving the updated params rounded to
+                                  nearest even (entries may be NULL), or NULL */
+} fp8adam_options;
+
+/* fp8adam_create with options (fp8adam_create is this call with the options
+ * all off).  Returns INVALID_ARG for bad options. */
+int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tensors,
+                      const fp8adam_options* opts, fp8adam_ctx** out);
+
+typedef struct {
+  float lr, beta1, beta2, eps, weight_decay;
+  int64_t step;              /* 1-based */
+  float loss_scale;          /* gradients are divided by it (1: none; > 0) */
+  float max_norm;            /* <= 0: no clipping; else the global L2 norm of the
+                                unscaled gradients over all tensors is clipped to it */
+  int32_t skip_nonfinite;    /* non-zero: if any gradient is inf/NaN the whole step
+                                leaves every buffer untouched */
+} fp8adam_step_params;
+
+/* One step with per-step gradient handling.  When loss_scale != 1, max_norm >
+ * 0 or skip_nonfinite is set, a pre-pass over all gradients computes (in a
+ * fixed reduction order) sumsq = sum of g^2, the multiplier c = (1/loss_scale)
+ * * min(1, max_norm / (sqrt(sumsq)/loss_scale + 1e-6)) (double, rounded once
+ * to fp32; clip_grad_norm_'s formula) and the non-finite count; the step then
+ * uses g*c in place of g.  Asynchronous on cuda_stream. */
+int fp8adam_step_ex(fp8adam_ctx* ctx, const fp8adam_step_params* params,
+                    void* cuda_stream);
+
+/* Results of the last fp8adam_step_ex pre-pass: *grad_norm = the global L2
+ * norm of the unscaled gradients, *skipped = 1 if that step was skipped.
+ * Host outputs; waits for cuda_stream.  Zeros if no pre-pass ran. */
+int fp8adam_get_grad_info(fp8adam_ctx* ctx, double* grad_norm,
+                          uint32_t* skipped, void* cuda_stream);
+
 /* ---- device codec (verification entry points) -------------------------
  * impl 0 = hardware conversion (cvt.rn.satfinite.{e4m3x2,e5m2x2}.f32 /
  * cvt.rn.f16x2.{e4m3x2,e5m2x2}), impl 1 = integer/bit-manipulation path.

@@ -23,6 +23,16 @@ LIB = os.path.join(HERE, "liboracle_fp8adam.so")
 # Format identifiers of the oracle.
 E4M3, E5M2, FP32 = 0, 1, 2
 FLAG_JIT_EVERY_STEP = 2
+FLAG_UPDATE_FROM_STORED = 4
+FLAG_STOCHASTIC = 8
+
+
+class StepOpts(ctypes.Structure):
+    """Options of the extended step (mirrors ref_step_opts in the C source)."""
+    _fields_ = [("flags", ctypes.c_uint32), ("margin_m", ctypes.c_int32), ("margin_v", ctypes.c_int32),
+                ("hist_len", ctypes.c_int32), ("hist_m", ctypes.c_void_p), ("hist_v", ctypes.c_void_p),
+                ("seed", ctypes.c_uint64), ("tensor_index", ctypes.c_int32), ("grad_mult", ctypes.c_float),
+                ("skip", ctypes.c_int32), ("p_bf16", ctypes.c_void_p)]
 
 CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
           "-Wall", "-Wextra"]
@@ -67,6 +77,24 @@ def lib() -> ctypes.CDLL:
         L.ref_fp8adam_step_tensor.argtypes = [
             c_i64, vp, vp, vp, vp, vp, vp, vp, vp, c_int, c_int,
             c_f, c_f, c_f, c_f, c_f, c_i64, c_u32, vp]
+        L.ref_fp8adam_step_tensor_ex.restype = c_int
+        L.ref_fp8adam_step_tensor_ex.argtypes = [
+            c_i64, vp, vp, vp, vp, vp, vp, vp, vp, c_int, c_int,
+            c_f, c_f, c_f, c_f, c_f, c_i64, c_u32, ctypes.POINTER(StepOpts), vp]
+        L.ref_philox4x32_10.restype = None
+        L.ref_philox4x32_10.argtypes = [vp, vp, vp]
+        L.ref_sr_bits.restype = c_u32
+        L.ref_sr_bits.argtypes = [ctypes.c_uint64, ctypes.c_int32, c_i64, c_i64, c_int]
+        L.ref_encode_sr.restype = c_u32
+        L.ref_encode_sr.argtypes = [c_int, c_f, c_u32]
+        L.ref_f32_to_bf16.restype = ctypes.c_uint16
+        L.ref_f32_to_bf16.argtypes = [c_f]
+        L.ref_f32_to_bf16_array.restype = None
+        L.ref_f32_to_bf16_array.argtypes = [vp, c_i64, vp]
+        L.ref_grad_sumsq.restype = None
+        L.ref_grad_sumsq.argtypes = [ctypes.c_int32, vp, vp, vp, vp]
+        L.ref_grad_multiplier.restype = c_f
+        L.ref_grad_multiplier.argtypes = [ctypes.c_double, c_f, c_f]
     return _lib
 
 
@@ -107,6 +135,45 @@ def pow2scale(fmt: int, amax: float, s_prev: float, margin: int = 0) -> float:
     return float(lib().ref_pow2scale(fmt, amax, s_prev, margin))
 
 
+def philox4x32_10(ctr, key) -> list:
+    c = np.asarray(ctr, np.uint32)
+    k = np.asarray(key, np.uint32)
+    out = np.empty(4, np.uint32)
+    lib().ref_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return [int(x) for x in out]
+
+
+def sr_bits(seed: int, tensor: int, t: int, j: int, which: int) -> int:
+    return int(lib().ref_sr_bits(seed, tensor, t, j, which))
+
+
+def encode_sr(fmt: int, x: float, r: int) -> int:
+    return int(lib().ref_encode_sr(fmt, x, r))
+
+
+def f32_to_bf16(x) -> np.ndarray:
+    a = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(a.shape, np.uint16)
+    lib().ref_f32_to_bf16_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def grad_sumsq(grads) -> tuple:
+    """(exact sum of g^2 rounded to double, non-finite count) over a list of
+    bf16-bit numpy arrays."""
+    arrs = [np.ascontiguousarray(g, dtype=np.uint16) for g in grads]
+    n = np.array([a.size for a in arrs], np.int64)
+    ptrs = np.array([a.ctypes.data for a in arrs], np.uint64)
+    s = ctypes.c_double()
+    bad = ctypes.c_uint64()
+    lib().ref_grad_sumsq(len(arrs), _ptr(n), _ptr(ptrs), ctypes.addressof(s), ctypes.addressof(bad))
+    return s.value, bad.value
+
+
+def grad_multiplier(sumsq: float, loss_scale: float, max_norm: float) -> float:
+    return float(lib().ref_grad_multiplier(sumsq, loss_scale, max_norm))
+
+
 def step_constants(lr, beta1, beta2, eps, wd, t) -> np.ndarray:
     out = np.empty(8, np.float32)
     lib().ref_step_constants(lr, beta1, beta2, eps, wd, t, _ptr(out))
@@ -133,6 +200,30 @@ class TensorState:
         self.amax_m = np.array([amax_m], np.float32)
         self.amax_v = np.array([amax_v], np.float32)
         self.stats = np.zeros(2, np.uint64)
+
+    def step_ex(self, g_bits: np.ndarray, lr, beta1, beta2, eps, wd, t, flags=0, *, margin_m=0,
+                margin_v=0, hist_len=0, seed=0, tensor_index=0, grad_mult=1.0, skip=False,
+                want_bf16=False):
+        """The extended step (scaling/read-back variants, stochastic rounding,
+        gradient multiplier, bf16 param copy); state kept on this object."""
+        g = np.ascontiguousarray(g_bits, dtype=np.uint16)
+        assert g.size == self.p.size
+        if hist_len > 1 and getattr(self, "hist_m", None) is None:
+            self.hist_m = np.zeros(hist_len, np.float32)
+            self.hist_v = np.zeros(hist_len, np.float32)
+        self.p_bf16 = np.zeros(self.p.size, np.uint16) if want_bf16 else None
+        o = StepOpts(flags, margin_m, margin_v, hist_len,
+                     _ptr(self.hist_m) if hist_len > 1 else None,
+                     _ptr(self.hist_v) if hist_len > 1 else None,
+                     seed, tensor_index, grad_mult, 1 if skip else 0,
+                     _ptr(self.p_bf16) if want_bf16 else None)
+        rc = lib().ref_fp8adam_step_tensor_ex(
+            self.p.size, _ptr(self.p), _ptr(g), _ptr(self.m), _ptr(self.v),
+            _ptr(self.scale_m), _ptr(self.scale_v), _ptr(self.amax_m), _ptr(self.amax_v),
+            self.m_fmt, self.v_fmt, lr, beta1, beta2, eps, wd, t, flags, ctypes.byref(o),
+            _ptr(self.stats))
+        if rc != 0:
+            raise ValueError("oracle step rejected its arguments (rc=%d)" % rc)
 
     def step(self, g_bits: np.ndarray, lr, beta1, beta2, eps, wd, t, flags=0):
         g = np.ascontiguousarray(g_bits, dtype=np.uint16)

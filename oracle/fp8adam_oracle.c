@@ -358,3 +358,303 @@ int ref_fp8adam_step_tensor(int64_t n, float* p, const uint16_t* g, void* m,
   env_leave(guard);
   return 0;
 }
+
+/* ======================================================================== */
+/* Extensions (next rows of the build): scaling and read-back variants,      */
+/* stochastic rounding, fused loss-scale/clip multiplier, bf16 param copy.   */
+/* The default path above is untouched; ref_fp8adam_step_tensor_ex with all  */
+/* options off computes exactly what ref_fp8adam_step_tensor computes.       */
+/* ======================================================================== */
+
+/* Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
+ * easy as 1, 2, 3", SC 2011): ten rounds of two 32x32->64 multiplies, the key
+ * bumped by the Weyl constants between rounds. */
+void ref_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4]) {
+  uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+  uint32_t k0 = key_in[0], k1 = key_in[1];
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)c0;
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * (uint64_t)c2;
+    const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n1 = lo1, n2 = hi0 ^ c3 ^ k1, n3 = lo0;
+    c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+  }
+  out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* The 32 random bits of element j of tensor `tensor` at step t for moment
+ * `which` (0 = m, 1 = v): counter (j/2 low, j/2 high, tensor, t low), key
+ * (seed low, seed high); element j takes outputs 2*(j&1) + which. */
+uint32_t ref_sr_bits(uint64_t seed, int32_t tensor, int64_t t, int64_t j, int which) {
+  const uint64_t q = (uint64_t)j >> 1;
+  const uint32_t ctr[4] = {(uint32_t)q, (uint32_t)(q >> 32), (uint32_t)tensor, (uint32_t)t};
+  const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  uint32_t out[4];
+  ref_philox4x32_10(ctr, key, out);
+  return out[2 * (int)(j & 1) + which];
+}
+
+/* Stochastic rounding of x to the format: NaN -> 0x7F; |x| >= FMAX -> +-FMAX;
+ * otherwise, with lo <= |x| < hi the two neighbouring finite values, round up
+ * to hi iff r * (hi - lo) < (|x| - lo) * 2^32 (probability (|x|-lo)/(hi-lo)
+ * quantised to 2^-32); evaluated exactly in double. */
+uint32_t ref_encode_sr(int fmt, float x, uint32_t r) {
+  if (isnan(x)) return 0x7Fu;
+  const float* tab = g_table[fmt == ORC_E4M3 ? 0 : 1];
+  const uint32_t sign = signbit(x) ? 0x80u : 0u;
+  const double a = fabs((double)x);
+  const uint32_t cmax = fmt_maxcode(fmt);
+  if (a >= (double)tab[cmax]) return sign | cmax;
+  uint32_t lo = 0, hi = cmax;
+  while (hi - lo > 1) {
+    const uint32_t mid = (lo + hi) / 2;
+    if ((double)tab[mid] <= a) lo = mid; else hi = mid;
+  }
+  const double below = a - (double)tab[lo];                  /* exact */
+  const double gap = (double)tab[hi] - (double)tab[lo];      /* a power of two */
+  const int up = (double)r * gap < below * 4294967296.0;     /* both sides exact */
+  return sign | (up ? hi : lo);
+}
+
+/* bf16 nearest-even rounding of an fp32 value written from the definition:
+ * 8 significant bits, rint() (round half to even) on the scaled significand. */
+uint16_t ref_f32_to_bf16(float x) {
+  uint32_t u;
+  memcpy(&u, &x, 4);
+  if (isnan(x)) return (uint16_t)((u >> 16) | 0x0040u);  /* quiet NaN, sign kept */
+  if (isinf(x) || x == 0.0f) return (uint16_t)(u >> 16);
+  int e;
+  (void)frexp((double)x, &e);               /* x = fr * 2^e, |fr| in [0.5, 1) */
+  /* bf16 keeps 8 significant bits for normals; below 2^-126 the quantum is
+   * fixed at 2^-133 (subnormals) */
+  int q = e - 8;
+  if (q < -133) q = -133;
+  const double n = rint(ldexp((double)x, -q));             /* ties to even */
+  const double y = ldexp(n, q);
+  float yf = (float)y;                                      /* exact or overflow to inf */
+  uint32_t v;
+  memcpy(&v, &yf, 4);
+  return (uint16_t)(v >> 16);
+}
+
+/* Global gradient statistics of the fused unscale / clip pre-pass:
+ * *sumsq = the exact sum of g^2 over all tensors, rounded once to double
+ * (each bf16 g^2 is an integer times a power of two; they are summed in a
+ * fixed-point accumulator wide enough to be exact), *nonfinite = count of
+ * non-finite gradients. */
+#define ACC_LIMBS 12  /* 768 bits: g^2 spans 2^-266 .. 2^256, plus carry room */
+void ref_grad_sumsq(int32_t T, const int64_t* numel, const uint16_t* const* grads, double* sumsq,
+                    uint64_t* nonfinite) {
+  uint64_t acc[ACC_LIMBS] = {0};
+  uint64_t bad = 0;
+  for (int32_t i = 0; i < T; ++i) {
+    for (int64_t j = 0; j < numel[i]; ++j) {
+      const uint16_t b = grads[i][j];
+      const uint32_t ex = (b >> 7) & 0xFFu, man = b & 0x7Fu;
+      if (ex == 0xFFu) { ++bad; continue; }
+      /* |g| = sig * 2^(e2) with sig the integer significand (8 bits) */
+      const uint32_t sig = ex ? (man | 0x80u) : man;
+      const int e2 = ex ? (int)ex - 127 - 7 : -126 - 7;
+      if (!sig) continue;
+      /* g^2 = sig^2 * 2^(2*e2); bit position relative to 2^-280 */
+      const uint64_t sq = (uint64_t)sig * sig;
+      const int pos = 2 * e2 + 280;
+      const int limb = pos / 64, sh = pos % 64;
+      unsigned __int128 add = (unsigned __int128)sq << sh;
+      for (int k = limb; k < ACC_LIMBS && add; ++k) {
+        const unsigned __int128 s = (unsigned __int128)acc[k] + (uint64_t)add;
+        acc[k] = (uint64_t)s;
+        add = (add >> 64) + (s >> 64);
+      }
+    }
+  }
+  /* round the exact value once to double: sum the limbs from the most
+   * significant, using long double only to collect 64 bits at a time is not
+   * exact, so take the top 128 bits of the number and a sticky bit */
+  int top = ACC_LIMBS - 1;
+  while (top >= 0 && acc[top] == 0) --top;
+  if (top < 0) { *sumsq = 0.0; *nonfinite = bad; return; }
+  const int lead = 63 - __builtin_clzll(acc[top]);   /* leading bit inside limb */
+  const int msb = top * 64 + lead;                    /* absolute bit index */
+  /* 54 bits starting at msb (53 + guard) plus sticky */
+  uint64_t mant = 0;
+  int sticky = 0;
+  for (int b = 0; b < 54; ++b) {
+    const int bit = msb - b;
+    mant <<= 1;
+    if (bit >= 0) mant |= (acc[bit / 64] >> (bit % 64)) & 1u;
+  }
+  for (int bit = msb - 54; bit >= 0 && !sticky; --bit)
+    if ((acc[bit / 64] >> (bit % 64)) & 1u) sticky = 1;
+  /* mant has 54 bits: 53 kept + 1 guard */
+  uint64_t kept = mant >> 1;
+  const int guard = (int)(mant & 1u);
+  if (guard && (sticky || (kept & 1u))) ++kept;       /* round half to even */
+  *sumsq = ldexp((double)kept, msb - 52 - 280);
+  *nonfinite = bad;
+}
+
+/* The fused gradient multiplier of a step: c = (1/loss_scale) * min(1,
+ * max_norm / (norm + 1e-6)) with norm = sqrt(sumsq) / loss_scale (the L2 norm
+ * of the unscaled gradients, as clip_grad_norm_ defines it); max_norm <= 0
+ * disables clipping.  Computed in double, rounded once to fp32. */
+float ref_grad_multiplier(double sumsq, float loss_scale, float max_norm) {
+  const double inv = 1.0 / (double)loss_scale;
+  double coef = 1.0;
+  if (max_norm > 0.0f) {
+    const double norm = sqrt(sumsq) * inv;
+    coef = (double)max_norm / (norm + 1e-6);
+    if (coef > 1.0) coef = 1.0;
+  }
+  return (float)(inv * coef);
+}
+
+/* Extension flags. */
+#define ORC_FLAG_UPDATE_FROM_STORED 4u
+#define ORC_FLAG_STOCHASTIC 8u
+
+typedef struct {
+  uint32_t flags;         /* ORC_FLAG_* */
+  int32_t margin_m, margin_v;
+  int32_t hist_len;       /* > 1: scale from the max of the last hist_len amax */
+  float* hist_m;          /* [hist_len] this tensor's ring, slot (t-1) % hist_len */
+  float* hist_v;
+  uint64_t seed;          /* stochastic rounding */
+  int32_t tensor_index;   /* stochastic rounding counter */
+  float grad_mult;        /* g is multiplied by this first (1.0f: off) */
+  int32_t skip;           /* non-zero: leave everything untouched */
+  uint16_t* p_bf16;       /* optional: bf16 copy of the updated params */
+} ref_step_opts;
+
+static float hist_max(const float* h, int n) {
+  float a = 0.0f;
+  for (int k = 0; k < n; ++k) a = max_keep_nan(a, h[k]);
+  return a;
+}
+
+static uint32_t encode_opt(int fmt, float x, const ref_step_opts* o, int64_t t, int64_t j, int which) {
+  if (o->flags & ORC_FLAG_STOCHASTIC)
+    return ref_encode_sr(fmt, x, ref_sr_bits(o->seed, o->tensor_index, t, j, which));
+  return ref_encode(fmt, x);
+}
+
+int ref_fp8adam_step_tensor_ex(int64_t n, float* p, const uint16_t* g, void* m, void* v,
+                               float* scale_m, float* scale_v, float* amax_m, float* amax_v,
+                               int m_fmt, int v_fmt, float lr, float beta1, float beta2,
+                               float eps, float wd, int64_t t, uint32_t flags,
+                               const ref_step_opts* o, uint64_t* stats) {
+  if (n < 0 || t < 1 || !o) return -1;
+  if (m_fmt < 0 || m_fmt > 2 || v_fmt < 0 || v_fmt > 2) return -1;
+  if (o->hist_len > 1 && (!o->hist_m || !o->hist_v)) return -1;
+  if (n == 0 || o->skip) return 0;
+  fpenv_guard guard = env_enter();
+  const ref_consts c = make_consts(lr, beta1, beta2, eps, wd, t);
+  const float s_m = *scale_m, s_v = *scale_v;
+  const float inv_s_m = 1.0f / s_m;
+  const float inv_s_v = 1.0f / s_v;
+  const float gm = o->grad_mult;
+
+  float amax_in_m = *amax_m, amax_in_v = *amax_v;
+  if (o->hist_len > 1) {
+    amax_in_m = hist_max(o->hist_m, o->hist_len);
+    amax_in_v = hist_max(o->hist_v, o->hist_len);
+  }
+  const int jit = (t == 1) || (flags & ORC_FLAG_JIT_EVERY_STEP);
+  if (jit) {
+    float am = 0.0f, av = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+      const float g0 = bf16_to_f32(g[i]);
+      const float gi = g0 * gm;
+      const float mo = load_moment(m_fmt, m, i, inv_s_m);
+      const float vo = load_moment(v_fmt, v, i, inv_s_v);
+      const float t1 = c.b1 * mo;
+      const float t2 = c.omb1 * gi;
+      const float mn = t1 + t2;
+      const float gg = gi * gi;
+      const float t3 = c.b2 * vo;
+      const float t4 = c.omb2 * gg;
+      const float vn = t3 + t4;
+      am = max_keep_nan(am, fabsf(mn));
+      av = max_keep_nan(av, fabsf(vn));
+    }
+    amax_in_m = am;
+    amax_in_v = av;
+  }
+  const float s_m_new = m_fmt == ORC_FP32 ? s_m : ref_pow2scale(m_fmt, amax_in_m, s_m, o->margin_m);
+  const float s_v_new = v_fmt == ORC_FP32 ? s_v : ref_pow2scale(v_fmt, amax_in_v, s_v, o->margin_v);
+  const float inv_s_m_new = 1.0f / s_m_new;
+  const float inv_s_v_new = 1.0f / s_v_new;
+  const float fmax_m = m_fmt == ORC_FP32 ? INFINITY : ref_fmax(m_fmt);
+  const float fmax_v = v_fmt == ORC_FP32 ? INFINITY : ref_fmax(v_fmt);
+
+  float am = 0.0f, av = 0.0f;
+  uint64_t flushed = 0, saturated = 0;
+  for (int64_t i = 0; i < n; ++i) {
+    const float g0 = bf16_to_f32(g[i]);
+    const float gi = g0 * gm;
+    const float mo = load_moment(m_fmt, m, i, inv_s_m);
+    const float vo = load_moment(v_fmt, v, i, inv_s_v);
+    const float t1 = c.b1 * mo;
+    const float t2 = c.omb1 * gi;
+    const float mn = t1 + t2;
+    const float gg = gi * gi;
+    const float t3 = c.b2 * vo;
+    const float t4 = c.omb2 * gg;
+    const float vn = t3 + t4;
+    am = max_keep_nan(am, fabsf(mn));
+    av = max_keep_nan(av, fabsf(vn));
+    float mu = mn, vu = vn; /* the moments the update reads */
+    if (m_fmt == ORC_FP32) {
+      ((float*)m)[i] = mn;
+    } else {
+      const float xm = mn * s_m_new;
+      const uint32_t q = encode_opt(m_fmt, xm, o, t, i, 0);
+      ((uint8_t*)m)[i] = (uint8_t)q;
+      if (fabsf(xm) > fmax_m) ++saturated;
+      if (o->flags & ORC_FLAG_UPDATE_FROM_STORED) mu = ref_decode(m_fmt, q) * inv_s_m_new;
+    }
+    if (v_fmt == ORC_FP32) {
+      ((float*)v)[i] = vn;
+    } else {
+      const float xv = vn * s_v_new;
+      const uint32_t q = encode_opt(v_fmt, xv, o, t, i, 1);
+      ((uint8_t*)v)[i] = (uint8_t)q;
+      if (vn > 0.0f && (q & 0x7Fu) == 0u) ++flushed;
+      if (fabsf(xv) > fmax_v) ++saturated;
+      if (o->flags & ORC_FLAG_UPDATE_FROM_STORED) vu = ref_decode(v_fmt, q) * inv_s_v_new;
+    }
+    const float sq = sqrtf(vu);
+    const float den0 = sq * c.isbc2;
+    const float den = den0 + c.eps;
+    const float u = mu / den;
+    const float pd = p[i] * c.decay;
+    const float w = c.step_size * u;
+    p[i] = pd - w;
+    if (o->p_bf16) o->p_bf16[i] = ref_f32_to_bf16(p[i]);
+  }
+  *scale_m = s_m_new;
+  *scale_v = s_v_new;
+  *amax_m = am;
+  *amax_v = av;
+  if (o->hist_len > 1) {
+    o->hist_m[(t - 1) % o->hist_len] = am;
+    o->hist_v[(t - 1) % o->hist_len] = av;
+  }
+  if (stats) {
+    stats[0] += flushed;
+    stats[1] += saturated;
+  }
+  env_leave(guard);
+  return 0;
+}
+
+void ref_f32_to_bf16_array(const float* x, int64_t n, uint16_t* out) {
+  fpenv_guard g = env_enter();
+  for (int64_t i = 0; i < n; ++i) out[i] = ref_f32_to_bf16(x[i]);
+  env_leave(g);
+}

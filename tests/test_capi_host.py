@@ -80,3 +80,20 @@ def test_binding_raises_on_error_codes(L):
     with pytest.raises(capi.Fp8AdamError) as e:
         capi.fp8adam_step(0, 1e-3, 0.9, 0.95, 1e-8, 0.1, 1, 0)
     assert e.value.code == capi.ERR_INVALID_ARG
+
+
+def test_option_entry_points_reject_bad_arguments_on_host(L):
+    T = capi.fp8adam_tensor * 1
+    t = T(capi.fp8adam_tensor(8, 8, 8, 8, 16))
+    out = ctypes.c_void_p()
+    ok = dict(scale_m=8, scale_v=8, amax_m=8, amax_v=8, m_fmt=0, v_fmt=1)
+    assert L.fp8adam_create_ex(t, 1, None, ctypes.byref(out)) == capi.ERR_INVALID_ARG
+    for bad in (dict(margin_m=-1), dict(margin_v=65), dict(amax_history_len=4), dict(amax_history_len=2000),
+                dict(flags=64), dict(scale_v=0)):
+        o = capi.fp8adam_options(**{**ok, **bad})
+        assert L.fp8adam_create_ex(t, 1, ctypes.byref(o), ctypes.byref(out)) == capi.ERR_INVALID_ARG, bad
+    o = capi.fp8adam_options(**{**ok, "m_fmt": 7})
+    assert L.fp8adam_create_ex(t, 1, ctypes.byref(o), ctypes.byref(out)) == capi.ERR_UNSUPPORTED_FMT
+    sp = capi.fp8adam_step_params(1e-3, 0.9, 0.95, 1e-8, 0.1, 1, 1.0, 0.0, 0)
+    assert L.fp8adam_step_ex(None, ctypes.byref(sp), None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_get_grad_info(None, None, None, None) == capi.ERR_INVALID_ARG

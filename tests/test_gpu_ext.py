@@ -1,0 +1,161 @@
+"""The step's options through the C ABI (fp8adam_create_ex / fp8adam_step_ex)
+against the oracle's extended step, free-running from the same seeded state
+on the same seeded gradients.  Covered options:
+- scale margin and amax history;
+- update from stored moments;
+- stochastic rounding;
+- loss-scale removal, global-norm clipping and skip-on-non-finite;
+- the bf16 param copy."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_quantized_adam_b200 import FP8AdamW, workloads
+from gpu_harness import HP, bf16_host_bits
+
+pytestmark = pytest.mark.gpu
+
+SIZES = [70001, 4096, 33, 0, 3 * 4096 + 5, 200003]
+
+
+class ExtRun:
+    def __init__(self, cfg, sizes=SIZES, mf=oracle.E4M3, vf=oracle.E5M2, bf16=False, **opt):
+        self.specs = workloads.custom_layout(sizes)
+        dev = torch.device("cuda:0")
+        self.M = workloads.FlatModel(self.specs, dev, m_fp32=mf == oracle.FP32, v_fp32=vf == oracle.FP32)
+        M = self.M
+        workloads.init_params_into(self.specs, M.views(M.p), cfg)
+        self.cfg = cfg
+        self.sig = workloads.tensor_sigmas(self.specs, cfg)
+        self.bf16 = [torch.zeros(s.numel, dtype=torch.bfloat16, device=dev) for s in self.specs] if bf16 else None
+        self.opt_kw = opt
+        self.opt = FP8AdamW(M.views(M.p), M.views(M.g), m_fmt=mf, v_fmt=vf, m=M.views(M.m), v=M.views(M.v),
+                            scale_m=M.scale_m, scale_v=M.scale_v, amax_m=M.amax_m, amax_v=M.amax_v,
+                            param_bf16=self.bf16, **opt)
+        torch.cuda.synchronize()
+        self.ref = [oracle.TensorState(M.view(M.p, i).cpu().numpy(), mf, vf) for i in range(len(self.specs))]
+        self.t = 0
+        self.flags = ((oracle.FLAG_UPDATE_FROM_STORED if opt.get("update_from_stored") else 0)
+                      | (oracle.FLAG_STOCHASTIC if opt.get("stochastic_rounding") else 0))
+
+    def step(self, loss_scale=1.0, max_norm=0.0, skip_nonfinite=False, poison=None, fill=None):
+        self.t += 1
+        M = self.M
+        workloads.grads_into(self.specs, M.views(M.g), self.cfg, self.t, self.sig)
+        if fill is not None:  # tensor index -> a constant gradient value
+            for i, f in fill.items():
+                M.view(M.g, i).fill_(f)
+        if poison is not None:
+            M.g[poison] = float("inf")
+        self.opt.step(loss_scale=loss_scale, max_norm=max_norm, skip_nonfinite=skip_nonfinite)
+        grads = [bf16_host_bits(M.view(M.g, i)) for i in range(len(self.specs))]
+        gm, skip, norm = 1.0, False, None
+        if loss_scale != 1.0 or max_norm > 0 or skip_nonfinite:
+            sumsq, bad = oracle.grad_sumsq(grads)
+            gm = oracle.grad_multiplier(sumsq, loss_scale, max_norm)
+            skip = bool(skip_nonfinite and bad > 0)
+            norm = math.sqrt(sumsq) / loss_scale
+        for i, r in enumerate(self.ref):
+            r.step_ex(grads[i], HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], self.t,
+                      self.flags, margin_m=self.opt_kw.get("margin_m", 0), margin_v=self.opt_kw.get("margin_v", 0),
+                      hist_len=self.opt_kw.get("amax_history_len", 0), seed=self.opt_kw.get("seed", 0),
+                      tensor_index=i, grad_mult=gm, skip=skip, want_bf16=self.bf16 is not None)
+        return norm, skip
+
+    def compare(self):
+        torch.cuda.synchronize()
+        M = self.M
+        for i, r in enumerate(self.ref):
+            for name, got, exp in (("p", M.view(M.p, i), r.p), ("m", M.view(M.m, i), r.m), ("v", M.view(M.v, i), r.v)):
+                g = got.cpu().numpy()
+                assert (g.view(np.uint8) == exp.view(np.uint8)).all(), (i, name, np.flatnonzero(g != exp)[:5])
+            for name, arr, exp in (("scale_m", M.scale_m, r.scale_m), ("scale_v", M.scale_v, r.scale_v),
+                                   ("amax_m", M.amax_m, r.amax_m), ("amax_v", M.amax_v, r.amax_v)):
+                assert np.float32(arr[i].item()).view(np.uint32) == exp.view(np.uint32)[0], (i, name)
+            if self.bf16 is not None and r.p.size:
+                b = self.bf16[i].cpu().view(torch.int16).numpy().view(np.uint16)
+                assert (b == r.p_bf16).all(), (i, "bf16")
+            if getattr(r, "hist_m", None) is not None:
+                h = self.opt.hist_m[:, i].cpu().numpy()
+                assert (h.view(np.uint32) == r.hist_m.view(np.uint32)).all(), (i, "hist_m")
+
+
+def test_margin_and_amax_history():
+    r = ExtRun(41, margin_m=1, margin_v=2, amax_history_len=4)
+    for _ in range(9):
+        r.step()
+        r.compare()
+
+
+def test_margin_with_subnormal_amax():
+    """Gradients of 1e-21 make v ~5e-44 (an fp32 subnormal): its scale with a
+    large margin depends on the subnormal's exact exponent."""
+    r = ExtRun(48, margin_m=20, margin_v=30)
+    for _ in range(4):
+        r.step(fill={1: 1e-21})
+        r.compare()
+    assert 0 < float(r.M.amax_v[1]) < 1.2e-38
+
+
+@pytest.mark.parametrize("vf", [oracle.E5M2, oracle.E4M3], ids=["v5", "v4"])
+def test_update_from_stored_moments(vf):
+    r = ExtRun(42, vf=vf, update_from_stored=True)
+    for _ in range(5):
+        r.step()
+        r.compare()
+
+
+@pytest.mark.parametrize("fmts", [(oracle.E4M3, oracle.E5M2), (oracle.E5M2, oracle.E4M3)], ids=["m4v5", "m5v4"])
+def test_stochastic_rounding(fmts):
+    r = ExtRun(43, mf=fmts[0], vf=fmts[1], stochastic_rounding=True, seed=0x0123456789ABCDEF)
+    for _ in range(5):
+        r.step()
+        r.compare()
+
+
+def test_bf16_param_copy():
+    r = ExtRun(44, bf16=True)
+    for _ in range(3):
+        r.step()
+        r.compare()
+
+
+def test_loss_scale_clip_and_skip():
+    r = ExtRun(45)
+    for ls, mx in ((1024.0, 1.0), (1.0, 0.05), (65536.0, 0.0), (8.0, 1e-4)):
+        norm, skip = r.step(loss_scale=ls, max_norm=mx, skip_nonfinite=True)
+        r.compare()
+        gn, sk = r.opt.grad_info()
+        assert sk == 0 and math.isclose(gn, norm, rel_tol=1e-12)
+    # an inf gradient: the whole step is skipped on both sides
+    before = r.M.p.clone()
+    norm, skip = r.step(loss_scale=2.0, max_norm=1.0, skip_nonfinite=True, poison=123)
+    assert skip
+    r.compare()
+    assert r.opt.grad_info()[1] == 1
+    assert torch.equal(before, r.M.p)
+
+
+def test_prepass_only_equals_default_kernel():
+    """skip_nonfinite alone (multiplier 1, nothing skipped) runs the variant
+    kernels; the results equal the default step bit for bit."""
+    a = ExtRun(46)
+    b = ExtRun(46)
+    for _ in range(3):
+        a.step(skip_nonfinite=True)
+        b.step()
+    torch.cuda.synchronize()
+    for x in ("p", "m", "v", "scale_m", "scale_v", "amax_m", "amax_v"):
+        assert torch.equal(getattr(a.M, x).view(torch.uint8), getattr(b.M, x).view(torch.uint8)), x
+
+
+def test_options_with_fp32_moments_and_current_scaling():
+    r = ExtRun(47, mf=oracle.FP32, vf=oracle.E5M2, margin_v=1, stochastic_rounding=True, seed=5,
+               jit_every_step=True)
+    r.flags |= oracle.FLAG_JIT_EVERY_STEP
+    for _ in range(4):
+        r.step(loss_scale=4.0, max_norm=0.5)
+        r.compare()

@@ -1,0 +1,113 @@
+"""ZeRO-1 orchestration with world_size 2 on gloo (CPU).
+
+The sharded step's bookkeeping is what is tested here: the whole-tensor
+partition, rank-blocked flat buffers, reduce-scatter of the gradients,
+the step on owned tensors only, and the all-gather of the params.  The local
+step is the CPU oracle, a test stand-in for the CUDA kernels; the product's
+local step is FP8AdamW.  After three steps every rank's params must equal a
+single-process oracle run over all tensors on the summed gradients.
+"""
+import os
+import socket
+
+import numpy as np
+import torch
+import torch.multiprocessing as mp
+
+import oracle
+from fp8_quantized_adam_b200 import ranks, workloads, zero
+
+HP = workloads.HPARAMS
+SIZES = [70001, 4096, 33, 200003, 5000, 1, 0]
+
+
+def _bits(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+class OracleLocal:
+    """CPU stand-in for FP8AdamW over the owned tensors (views are updated in
+    place so the all-gather sees the new params)."""
+
+    def __init__(self, p_views, g_views, **kw):
+        self.p, self.g = p_views, g_views
+        self.st = [oracle.TensorState(p.numpy(), oracle.E4M3, oracle.E5M2) for p in p_views]
+        self.t = 0
+
+    def step(self, loss_scale=1.0, **kw):
+        self.t += 1
+        c = oracle.grad_multiplier(0.0, loss_scale, 0.0)
+        for p, g, st in zip(self.p, self.g, self.st):
+            st.step_ex(_bits(g), HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], self.t,
+                       grad_mult=c)
+            p.copy_(torch.from_numpy(st.p))
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank),
+                      LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+
+    ranks.init("gloo", timeout_s=60)
+    specs = workloads.custom_layout(SIZES)
+    L = zero.ShardLayout([s.numel for s in specs], world)
+    params = torch.zeros(L.total)
+    workloads.init_params_into(specs, L.views(params), 51)  # identical on every rank
+    p0 = params.clone()
+    grads = torch.zeros(L.total, dtype=torch.bfloat16)
+    opt = zero.ZeroFP8AdamW(L, params, grads, make_local=OracleLocal)
+    sig = workloads.tensor_sigmas(specs, 51)
+    reduced = []
+    for t in range(1, 4):
+        workloads.grads_into(specs, L.views(grads), 51 + 100 * rank, t, sig)  # each rank its own grads
+        opt.step()
+        full = torch.zeros(L.total, dtype=torch.bfloat16)
+        dist.all_gather_into_tensor(full, opt.g_block)
+        reduced.append(full)
+    if rank == 0:
+        # single process: every tensor, the summed gradients, the same average
+        c = oracle.grad_multiplier(0.0, float(world), 0.0)
+        ref = [oracle.TensorState(v.numpy(), oracle.E4M3, oracle.E5M2) for v in L.views(p0)]
+        for t, full in enumerate(reduced, start=1):
+            for st, g in zip(ref, L.views(full)):
+                st.step_ex(_bits(g), HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], t,
+                           grad_mult=c)
+        ok = all((v.numpy().view(np.uint32) == st.p.view(np.uint32)).all() for v, st in zip(L.views(params), ref))
+        q.put(("rank0", ok, [len(p) for p in L.parts]))
+    else:
+        q.put(("rank1", True, None))
+    ranks.finish()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_zero1_world2_matches_single_process_oracle():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    res = dict((k, (ok, parts)) for k, ok, parts in (q.get(timeout=300), q.get(timeout=300)))
+    for p in ps:
+        p.join(timeout=120)
+    ok, parts = res["rank0"]
+    assert ok
+    assert sum(parts) == len(SIZES) and min(parts) >= 1  # both ranks own tensors
+
+
+def test_shard_layout_blocks():
+    specs = workloads.layout("llama2_7b")
+    for world in (1, 2, 8):
+        L = zero.ShardLayout([s.numel for s in specs], world)
+        assert L.total == L.block * world
+        starts = sorted((L.flat_index(i), i) for i in range(len(specs)))
+        for (a, i), (b, _) in zip(starts, starts[1:]):
+            assert a + specs[i].numel <= b  # no overlap
+        for i in range(len(specs)):
+            assert L.flat_index(i) % zero.ALIGN == 0
+            assert L.offset[i] + specs[i].numel <= L.block
