@@ -63,7 +63,7 @@ def hbm_peak():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -78,7 +78,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except Exception:
@@ -229,7 +229,8 @@ def our_arm(args):
     sig = workloads.tensor_sigmas(specs, cfg)
     workloads.grads_into(specs, model.views(model.g), seed, 1, sig)
     opt = FP8AdamW(model.views(model.p), model.views(model.g), m=model.views(model.m), v=model.views(model.v),
-                   scale_m=model.scale_m, scale_v=model.scale_v, amax_m=model.amax_m, amax_v=model.amax_v)
+                   scale_m=model.scale_m, scale_v=model.scale_v, amax_m=model.amax_m, amax_v=model.amax_v,
+                   chunk_elems=args.chunk_elems)
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -388,6 +389,7 @@ def main():
     ap.add_argument("--workload", default="llama2_7b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--chunk-elems", type=int, default=0, help="elements per CTA (0: chosen by the library)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--report", choices=["ablation"], default=None,

@@ -1,9 +1,9 @@
 // fp8adam_capi.cu -- the C ABI declared in include/fp8adam.h.
 //
 // Host side of the FP8-moment AdamW step: argument validation, the device
-// tensor table and tile prefix, persistent grid sizing, per-step constants
-// (computed in double, rounded once to fp32) and kernel dispatch over the
-// (m format, v format, stats) variants.
+// tensor and chunk tables, per-step constants (computed in double, rounded
+// once to fp32) and kernel dispatch over the (m format, v format, stats)
+// variants, the option kernels and the gradient pre-pass.
 // The kernels are in fp8adam_step.cuh; the codec in fp8_codec.cuh.
 
 #include <cuda_runtime.h>
@@ -158,21 +158,18 @@ struct fp8adam_ctx {
   int32_t T = 0;
   int32_t m_fmt = 0, v_fmt = 0;
   uint32_t flags = 0;
-  int32_t total_units = 0;                        // work units of the schedule
-  int32_t step_grid = 0, step_tiles_per_cta = 0;  // grid of the step kernel
-  int32_t amax_grid = 0, amax_tiles_per_cta = 0;  // and of the pre-pass
+  int32_t total_units = 0;  // chunks of the whole list = grid of every per-step kernel
+  int32_t chunk_elems = 0;  // elements per chunk
   float *scale_m = nullptr, *scale_v = nullptr, *amax_m = nullptr, *amax_v = nullptr;
   TensorDesc* d_tensors = nullptr;
-  int32_t* d_unit_begin = nullptr;
-  Chunk* d_chunks = nullptr;  // chunk schedule
+  Chunk* d_chunks = nullptr;
   // options of fp8adam_create_ex
   int32_t margin_m = 0, margin_v = 0, hist_len = 0;
   float *hist_m = nullptr, *hist_v = nullptr;
   uint64_t seed = 0;
   uint16_t** d_bf16 = nullptr;  // device [T] bf16 outputs, or null
   bool ext = false;             // any option on: the variant kernels run
-  int32_t ext_grid = 0, ext_tiles_per_cta = 0, aext_grid = 0, aext_tiles_per_cta = 0;
-  // gradient pre-pass of fp8adam_step_ex: [step_grid] partials, non-finite
+  // gradient pre-pass of fp8adam_step_ex: [chunks] partials, non-finite
   // count, multiplier, skip flag, norm
   double* d_partial = nullptr;
   unsigned long long* d_nonfinite = nullptr;
@@ -186,7 +183,6 @@ struct fp8adam_ctx {
 static void free_ctx(fp8adam_ctx* c) {
   if (!c) return;
   cudaFree(c->d_tensors);
-  cudaFree(c->d_unit_begin);
   cudaFree(c->d_chunks);
   cudaFree(c->d_bf16);
   cudaFree(c->d_partial);
@@ -197,30 +193,6 @@ static void free_ctx(fp8adam_ctx* c) {
   cudaFree(c->d_state);
   cudaFree(c->d_stats);
   delete c;
-}
-
-// Grid of a kernel over the context's work units.  One CTA per chunk, or
-// (persistent schedule) every SM filled with as many CTAs as can be resident,
-// each taking a contiguous, equal range of tiles (no CTA without work).
-static int size_grid(const fp8adam_ctx* c, const void* kernel, int32_t* grid, int32_t* per_cta) {
-#if !FP8ADAM_PERSISTENT
-  (void)kernel;
-  *grid = c->total_units > 0 ? c->total_units : 1;
-  *per_cta = 1;
-  return FP8ADAM_OK;
-#endif
-  int sms = 0, occ = 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, 0) != cudaSuccess) {
-    cudaGetLastError();
-    return FP8ADAM_ERR_CUDA;
-  }
-  const int64_t slots = (int64_t)sms * (occ > 0 ? occ : 1);
-  const int64_t tiles = c->total_units > 0 ? c->total_units : 1;
-  const int64_t per = (tiles + slots - 1) / slots;
-  *per_cta = (int32_t)per;
-  *grid = (int32_t)((tiles + per - 1) / per);
-  return FP8ADAM_OK;
 }
 
 extern "C" int fp8adam_create(const fp8adam_tensor* tensors, int32_t num_tensors, float* scale_m,
@@ -255,45 +227,60 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
   if (flags & ~(FP8ADAM_FLAG_STATS | FP8ADAM_FLAG_JIT_EVERY_STEP | FP8ADAM_FLAG_UPDATE_FROM_STORED |
                 FP8ADAM_FLAG_STOCHASTIC_ROUNDING))
     return FP8ADAM_ERR_INVALID_ARG;
+  if (opts->chunk_elems < 0 || opts->chunk_elems > kChunk || opts->chunk_elems % kTile != 0)
+    return FP8ADAM_ERR_INVALID_ARG;
   if (opts->margin_m < 0 || opts->margin_m > 64 || opts->margin_v < 0 || opts->margin_v > 64 ||
       opts->amax_history_len < 0 || opts->amax_history_len > 1024 ||
       (opts->amax_history_len > 1 && (!opts->amax_history_m || !opts->amax_history_v)))
     return FP8ADAM_ERR_INVALID_ARG;
 
   std::vector<TensorDesc> desc((size_t)num_tensors);
-  std::vector<int32_t> unit_begin((size_t)num_tensors + 1);
-  int64_t total_units = 0;
   for (int32_t i = 0; i < num_tensors; ++i) {
     const fp8adam_tensor& t = tensors[i];
     if (t.numel < 0) return FP8ADAM_ERR_INVALID_ARG;
     if (t.numel > 0 && (!t.param || !t.grad || !t.m || !t.v)) return FP8ADAM_ERR_INVALID_ARG;
-    const int64_t nt = (t.numel + kUnit - 1) / kUnit;
-    unit_begin[(size_t)i] = (int32_t)total_units;
-    total_units += nt;
-    if (total_units > INT32_MAX / 2) return FP8ADAM_ERR_INVALID_ARG;
+  }
+  int dev = -1, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FP8ADAM_ERR_CUDA;
+  }
+  auto count_chunks = [&](int64_t ce) {
+    int64_t n = 0;
+    for (int32_t i = 0; i < num_tensors; ++i) n += (tensors[i].numel + ce - 1) / ce;
+    return n;
+  };
+  // chunk length: the largest that keeps >= 8 waves of resident CTAs (4 per
+  // SM), so the last partial wave costs little; never below 16384
+  int64_t chunk = opts->chunk_elems;
+  if (chunk == 0) {
+    const int64_t want = (int64_t)sms * 4 * 8;
+    chunk = kChunk;
+    while (chunk > 16384 && count_chunks(chunk) < want) chunk /= 2;
+  }
+  const int64_t total_units = count_chunks(chunk);
+  if (total_units > INT32_MAX / 2) return FP8ADAM_ERR_INVALID_ARG;
+  std::vector<Chunk> chunks;
+  chunks.reserve((size_t)total_units);
+  for (int32_t i = 0; i < num_tensors; ++i) {
+    const fp8adam_tensor& t = tensors[i];
     TensorDesc& d = desc[(size_t)i];
     d.p = t.param;
     d.g = t.grad;
     d.m = t.m;
     d.v = t.v;
     d.numel = t.numel;
-    d.nunits = (int32_t)nt;
+    d.nunits = (int32_t)((t.numel + chunk - 1) / chunk);
     d.aligned = aligned16(t.param) && aligned16(t.grad) && aligned16(t.m) && aligned16(t.v);
+    for (int64_t st = 0; st < t.numel; st += chunk)
+      chunks.push_back(Chunk{i, (int32_t)(t.numel - st < chunk ? t.numel - st : chunk), st});
   }
-  unit_begin[(size_t)num_tensors] = (int32_t)total_units;
-  std::vector<Chunk> chunks;
-#if !FP8ADAM_PERSISTENT
-  chunks.reserve((size_t)total_units);
-  for (int32_t i = 0; i < num_tensors; ++i)
-    for (int64_t st = 0; st < tensors[i].numel; st += kChunk) chunks.push_back(Chunk{i, 0, st});
-#endif
 
   fp8adam_ctx* c = new (std::nothrow) fp8adam_ctx();
   if (!c) return FP8ADAM_ERR_OOM;
-  if (cudaGetDevice(&c->device) != cudaSuccess) {
-    delete c;
-    return FP8ADAM_ERR_CUDA;
-  }
+  c->device = dev;
+  c->chunk_elems = (int32_t)chunk;
   c->T = num_tensors;
   c->m_fmt = m_fmt;
   c->v_fmt = v_fmt;
@@ -313,7 +300,6 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
            c->margin_v || c->hist_len || opts->param_bf16;
   const size_t T = (size_t)num_tensors;
   if (cudaMalloc(&c->d_tensors, T * sizeof(TensorDesc)) != cudaSuccess ||
-      cudaMalloc(&c->d_unit_begin, (T + 1) * sizeof(int32_t)) != cudaSuccess ||
       cudaMalloc(&c->d_chunks, (chunks.empty() ? 1 : chunks.size()) * sizeof(Chunk)) != cudaSuccess ||
       cudaMalloc(&c->d_state, 5 * T * sizeof(uint32_t)) != cudaSuccess ||
       cudaMalloc(&c->d_stats, 2 * sizeof(unsigned long long)) != cudaSuccess) {
@@ -322,8 +308,6 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
     return FP8ADAM_ERR_OOM;
   }
   if (cudaMemcpy(c->d_tensors, desc.data(), T * sizeof(TensorDesc), cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy(c->d_unit_begin, unit_begin.data(), (T + 1) * sizeof(int32_t), cudaMemcpyHostToDevice) !=
-          cudaSuccess ||
       (!chunks.empty() &&
        cudaMemcpy(c->d_chunks, chunks.data(), chunks.size() * sizeof(Chunk), cudaMemcpyHostToDevice) != cudaSuccess) ||
       cudaMemset(c->d_state, 0, 5 * T * sizeof(uint32_t)) != cudaSuccess ||
@@ -333,19 +317,8 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
     free_ctx(c);
     return FP8ADAM_ERR_CUDA;
   }
-  const bool stats = (flags & FP8ADAM_FLAG_STATS) != 0;
-  if (size_grid(c, (const void*)pick_step(m_fmt, v_fmt, stats), &c->step_grid, &c->step_tiles_per_cta) !=
-          FP8ADAM_OK ||
-      size_grid(c, (const void*)pick_amax(m_fmt, v_fmt), &c->amax_grid, &c->amax_tiles_per_cta) != FP8ADAM_OK ||
-      size_grid(c, (const void*)pick_ext(m_fmt, v_fmt, stats), &c->ext_grid, &c->ext_tiles_per_cta) !=
-          FP8ADAM_OK ||
-      size_grid(c, (const void*)pick_amax_ext(m_fmt, v_fmt), &c->aext_grid, &c->aext_tiles_per_cta) !=
-          FP8ADAM_OK) {
-    free_ctx(c);
-    return FP8ADAM_ERR_CUDA;
-  }
   // gradient pre-pass buffers (partials over the step grid) and options
-  if (cudaMalloc(&c->d_partial, (size_t)(c->step_grid > 0 ? c->step_grid : 1) * sizeof(double)) != cudaSuccess ||
+  if (cudaMalloc(&c->d_partial, (size_t)(c->total_units > 0 ? c->total_units : 1) * sizeof(double)) != cudaSuccess ||
       cudaMalloc(&c->d_nonfinite, sizeof(unsigned long long)) != cudaSuccess ||
       cudaMalloc(&c->d_grad_mult, sizeof(float)) != cudaSuccess ||
       cudaMalloc(&c->d_skip, sizeof(uint32_t)) != cudaSuccess ||
@@ -400,10 +373,8 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
   uint32_t* jit_m = ctx->d_state + 2 * T;
   uint32_t* jit_v = ctx->d_state + 3 * T;
   a.tensors = ctx->d_tensors;
-  a.unit_begin = ctx->d_unit_begin;
   a.chunks = ctx->d_chunks;
   a.num_tensors = ctx->T;
-  a.total_tiles = ctx->total_units;
   a.scale_m = ctx->scale_m;
   a.scale_v = ctx->scale_v;
   a.amax_m = ctx->amax_m;
@@ -413,7 +384,7 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
   a.acc_m = acc_m;
   a.acc_v = acc_v;
 
-  const dim3 block(kThreads);
+  const dim3 block(kThreads), grid((unsigned)ctx->total_units);
   const bool jit = p.step == 1 || (ctx->flags & FP8ADAM_FLAG_JIT_EVERY_STEP);
   const bool stats = (ctx->flags & FP8ADAM_FLAG_STATS) != 0;
   if (!ext) {
@@ -424,8 +395,7 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
       pre.acc_v = jit_v;
       pre.amax_in_m = nullptr;
       pre.amax_in_v = nullptr;
-      pre.tiles_per_cta = ctx->amax_tiles_per_cta;
-      pick_amax(ctx->m_fmt, ctx->v_fmt)<<<dim3((unsigned)ctx->amax_grid), block, 0, st>>>(pre);
+      pick_amax(ctx->m_fmt, ctx->v_fmt)<<<grid, block, 0, st>>>(pre);
       g_launches.fetch_add(1, std::memory_order_relaxed);
       a.amax_in_m = jit_m;
       a.amax_in_v = jit_v;
@@ -433,8 +403,7 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
       a.amax_in_m = reinterpret_cast<const uint32_t*>(ctx->amax_m);
       a.amax_in_v = reinterpret_cast<const uint32_t*>(ctx->amax_v);
     }
-    a.tiles_per_cta = ctx->step_tiles_per_cta;
-    pick_step(ctx->m_fmt, ctx->v_fmt, stats)<<<dim3((unsigned)ctx->step_grid), block, 0, st>>>(a);
+    pick_step(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(a);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return last_error();
   }
@@ -455,13 +424,10 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
   e.skip = nullptr;
   e.p_bf16 = ctx->d_bf16;
   if (prepass) {
-    StepArgs g = a;
-    g.tiles_per_cta = ctx->step_tiles_per_cta;
     if (cudaMemsetAsync(ctx->d_nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)
       return FP8ADAM_ERR_CUDA;
-    fp8adam_gradnorm_partial_kernel<<<dim3((unsigned)ctx->step_grid), block, 0, st>>>(g, ctx->d_partial,
-                                                                                      ctx->d_nonfinite);
-    fp8adam_gradnorm_finalize_kernel<<<1, block, 0, st>>>(ctx->d_partial, ctx->step_grid, ctx->d_nonfinite,
+    fp8adam_gradnorm_partial_kernel<<<grid, block, 0, st>>>(a, ctx->d_partial, ctx->d_nonfinite);
+    fp8adam_gradnorm_finalize_kernel<<<1, block, 0, st>>>(ctx->d_partial, ctx->total_units, ctx->d_nonfinite,
                                                           p.loss_scale, p.max_norm, p.skip_nonfinite,
                                                           ctx->d_grad_mult, ctx->d_skip, ctx->d_norm);
     g_launches.fetch_add(2, std::memory_order_relaxed);
@@ -476,8 +442,7 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
     pre.s.acc_v = jit_v;
     pre.s.amax_in_m = nullptr;
     pre.s.amax_in_v = nullptr;
-    pre.s.tiles_per_cta = ctx->aext_tiles_per_cta;
-    pick_amax_ext(ctx->m_fmt, ctx->v_fmt)<<<dim3((unsigned)ctx->aext_grid), block, 0, st>>>(pre);
+    pick_amax_ext(ctx->m_fmt, ctx->v_fmt)<<<grid, block, 0, st>>>(pre);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     a.amax_in_m = jit_m;
     a.amax_in_v = jit_v;
@@ -485,9 +450,8 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
     a.amax_in_m = reinterpret_cast<const uint32_t*>(ctx->amax_m);
     a.amax_in_v = reinterpret_cast<const uint32_t*>(ctx->amax_v);
   }
-  a.tiles_per_cta = ctx->ext_tiles_per_cta;
   e.s = a;
-  pick_ext(ctx->m_fmt, ctx->v_fmt, stats)<<<dim3((unsigned)ctx->ext_grid), block, 0, st>>>(e);
+  pick_ext(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return last_error();
 }

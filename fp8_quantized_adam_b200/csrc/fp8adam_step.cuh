@@ -9,16 +9,18 @@
 //
 // Design for B200: the step is a pure HBM stream (read p 4 B, g 2 B, m 1 B,
 // v 1 B; write p 4 B, m 1 B, v 1 B per element).  One launch covers a whole
-// parameter list.  The list is cut into tiles of kTile elements (a tensor's
-// last tile may be short); a persistent grid of (SMs x resident CTAs) CTAs
-// takes contiguous, equal ranges of the global tile sequence.  Within a tile
-// each thread moves 16 elements with 16-byte loads and stores (4 x p, 2 x g,
-// 1 x m, 1 x v), streaming cache hints, all fp32 arithmetic as single IEEE
-// operations (no FMA contraction), hardware cvt for the FP8 conversions.  A
-// CTA keeps the running amax of the tensor it is in, and flushes it once per
-// tensor segment (warp redux, one atomicMax per moment); the CTA whose flush
-// completes a tensor's tile count publishes its amax and scale, so a step is
-// a single kernel (plus an amax pre-pass at step 1).
+// parameter list through a chunk table: CTA b handles chunk b, a run of
+// elements of one tensor (the chunk length is chosen per parameter list so
+// the grid has many waves; up to kChunk), 4 CTAs of 256 threads resident per
+// SM (64 registers).  Each thread moves 16 elements per iteration with 16-byte
+// loads and stores (4 x p, 2 x g, 1 x m, 1 x v), streaming cache hints, all
+// fp32 arithmetic as single IEEE operations (no FMA contraction), hardware
+// cvt for the FP8 conversions.  The new amax of the chunk is reduced with a
+// NaN-keeping max, a warp redux and one atomicMax per moment; the CTA that
+// completes a tensor's last chunk (per-tensor counter) publishes its amax and
+// scale, so a step is a single kernel (plus an amax pre-pass at step 1).
+// (Measured on the 7B-shaped layout: within 2% of a kernel with the same
+// loads and stores and no arithmetic.)
 #pragma once
 
 #include <stdint.h>
@@ -30,7 +32,7 @@ namespace fp8adam {
 constexpr int kThreads = 256;
 constexpr int kVec = 16;                     // elements per thread per tile
 constexpr int kTile = kThreads * kVec;       // 4096 elements per tile
-constexpr int64_t kChunk = 16 * (int64_t)kTile;  // 65536: work unit of the allocation-free path
+constexpr int64_t kChunk = 32 * (int64_t)kTile;  // 131072: the largest chunk (one CTA's work)
 
 // resident CTAs per SM the step kernel is built for (register budget): FP8
 // moments fit 64 registers per thread (4 x 256 threads), fp32 moments 128
@@ -45,15 +47,14 @@ struct TensorDesc {
   void* m;
   void* v;
   int64_t numel;
-  int32_t nunits;   // work units of the tensor (tiles of the step kernel, chunks
-                    // of the allocation-free path)
+  int32_t nunits;   // chunks of the tensor
   int32_t aligned;  // all four buffers 16-byte aligned
 };
 
-// One chunk of the chunk schedule: kChunk elements of a tensor from `start`.
+// One chunk: `len` elements of tensor `tensor` from `start` (one CTA's work).
 struct Chunk {
   int32_t tensor;
-  int32_t pad;
+  int32_t len;
   int64_t start;
 };
 
@@ -63,11 +64,8 @@ struct StepConsts {
 
 struct StepArgs {
   const TensorDesc* tensors;     // [T]
-  const int32_t* unit_begin;     // [T+1] first work unit (chunk or tile) of each tensor
-  const Chunk* chunks;           // chunk schedule: [total units] tensor and start of each chunk
+  const Chunk* chunks;           // [chunks] tensor and start of each chunk (one per CTA)
   int32_t num_tensors;
-  int32_t total_tiles;           // persistent schedule: tiles of the whole list
-  int32_t tiles_per_cta;         // persistent schedule: contiguous range of each CTA
   float* scale_m;            // [T] in: decode scale; out: encode scale of this step
   float* scale_v;
   float* amax_m;             // [T] out: max |m| of this step
@@ -132,19 +130,10 @@ __device__ __forceinline__ float update(const StepConsts& c, float p, float m, f
 
 __device__ __forceinline__ uint32_t umax(uint32_t a, uint32_t b) { return a > b ? a : b; }
 // max that returns NaN if either input is NaN (the canonical, positive NaN)
-#ifndef FP8ADAM_AMAX_INT
-#define FP8ADAM_AMAX_INT 0
-#endif
 __device__ __forceinline__ float fmax_nan(float a, float b) {
-#if FP8ADAM_AMAX_INT
-  // both non-negative or NaN: integer max of the bits keeps NaN (its bits
-  // exceed those of inf)
-  return __uint_as_float(umax(__float_as_uint(a), __float_as_uint(b) & 0x7FFFFFFFu));
-#else
   float d;
   asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
   return d;
-#endif
 }
 // |x| as ordered bits: integer max over them is a float max that keeps NaN
 __device__ __forceinline__ uint32_t abs_bits(float x) { return __float_as_uint(x) & 0x7FFFFFFFu; }
@@ -384,48 +373,14 @@ __device__ __forceinline__ void run_segment(const StepArgs& a, int ti, int64_t e
 }
 
 // ------------------------------------------------------------ the schedule
-// How a launch's CTAs cover the parameter list.  f(ti, e0, e1, units) is
-// called for each segment (an element range [e0, e1) of tensor ti standing
-// for `units` work units) of this CTA, in order.
-#ifndef FP8ADAM_PERSISTENT
-#define FP8ADAM_PERSISTENT 0
-#endif
-#if FP8ADAM_PERSISTENT
-// persistent grid: CTA b takes the contiguous tile range [b*tiles_per_cta,
-// (b+1)*tiles_per_cta) of the whole list; work units are tiles (kTile)
-constexpr int64_t kUnit = kTile;
+// One CTA per chunk (a multiple of kTile elements of one tensor, chosen per
+// context; a tensor's last chunk may be short).  f(ti, e0, e1, units) runs
+// the chunk as the element range [e0, e1) of tensor ti, one work unit.
 template <typename F>
 __device__ __forceinline__ void for_each_segment(const StepArgs& a, F&& f) {
-  const int32_t g0 = (int32_t)blockIdx.x * a.tiles_per_cta;
-  const int32_t g1 = min(g0 + a.tiles_per_cta, a.total_tiles);
-  if (g0 >= g1) return;
-  int lo = 0, hi = a.num_tensors;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (a.unit_begin[mid] <= g0) lo = mid; else hi = mid;
-  }
-  int ti = lo;
-  int32_t gt = g0;
-  while (gt < g1) {
-    while (a.unit_begin[ti + 1] <= gt) ++ti;  // skip empty tensors
-    const int32_t tb = a.unit_begin[ti];
-    const int32_t seg_end = min(a.unit_begin[ti + 1], g1);
-    f(ti, (int64_t)(gt - tb) * kTile, min((int64_t)(seg_end - tb) * kTile, a.tensors[ti].numel),
-      (uint32_t)(seg_end - gt));
-    __syncthreads();  // shared reduction buffers are reused by the next segment
-    gt = seg_end;
-    ++ti;
-  }
+  const Chunk ch = a.chunks[blockIdx.x];  // one 16-byte load: tensor, length, start
+  f(ch.tensor, ch.start, ch.start + ch.len, 1u);
 }
-#else
-// one CTA per chunk: work units are chunks of kChunk elements of one tensor
-constexpr int64_t kUnit = kChunk;
-template <typename F>
-__device__ __forceinline__ void for_each_segment(const StepArgs& a, F&& f) {
-  const Chunk ch = a.chunks[blockIdx.x];  // one 16-byte load: the tensor and the start
-  f(ch.tensor, ch.start, min(ch.start + kChunk, a.tensors[ch.tensor].numel), 1u);
-}
-#endif
 
 template <int MF, int VF, bool STATS, bool WRITE>
 __device__ __forceinline__ void step_body(const StepArgs& a) {

@@ -47,7 +47,7 @@ class FP8AdamW:
                  jit_every_step: bool = False, margin_m: int = 0, margin_v: int = 0,
                  amax_history_len: int = 0, update_from_stored: bool = False,
                  stochastic_rounding: bool = False, seed: int = 0,
-                 param_bf16: Optional[List[torch.Tensor]] = None):
+                 param_bf16: Optional[List[torch.Tensor]] = None, chunk_elems: int = 0):
         if len(params) == 0 or len(params) != len(grads):
             raise ValueError("need matching, non-empty param and grad lists")
         self.params, self.grads = list(params), list(grads)
@@ -98,7 +98,8 @@ class FP8AdamW:
                                     self.amax_history_len,
                                     self.hist_m.data_ptr() if self.hist_m is not None else None,
                                     self.hist_v.data_ptr() if self.hist_v is not None else None,
-                                    seed, ctypes.cast(bf16_arr, ctypes.c_void_p) if bf16_arr is not None else None)
+                                    seed, ctypes.cast(bf16_arr, ctypes.c_void_p) if bf16_arr is not None else None,
+                                    chunk_elems)
         with torch.cuda.device(dev):
             self.ctx = capi.fp8adam_create_ex(arr, T, opts)
         self.device = dev

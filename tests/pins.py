@@ -15,14 +15,12 @@ from __future__ import annotations
 
 import math
 import os
-import re
 
 import numpy as np
 import torch
 
 E4M3, E5M2, FP32 = 0, 1, 2
 FMAX = {E4M3: 448.0, E5M2: 57344.0}
-EMAX = {E4M3: 8, E5M2: 15}
 TORCH_DT = {E4M3: torch.float8_e4m3fn, E5M2: torch.float8_e5m2}
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 

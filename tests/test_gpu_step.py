@@ -8,7 +8,6 @@ import pytest
 import torch
 
 import oracle
-import pins
 from fp8_quantized_adam_b200 import FP8AdamW, capi, workloads
 from gpu_harness import HP, Run, bf16_host_bits
 
@@ -78,10 +77,12 @@ def test_current_scaling_every_step():
 
 
 def test_edge_sizes_and_misaligned_views():
-    """Sizes around the 16-element vector, the 4096-element CTA tile and the
-    65536-element chunk, an empty tensor, and tensors whose buffers are
-    offset by one element (element-by-element path)."""
-    sizes = [0, 1, 15, 16, 17, 4095, 4096, 4097, 65535, 65536, 65537, 3 * 65536 + 4099]
+    """Sizes around the 16-element vector, the 4096-element tile and the
+    chunk lengths the library picks (16384 .. 131072), an empty tensor, and
+    tensors whose buffers are offset by one element (element-by-element
+    path)."""
+    sizes = [0, 1, 15, 16, 17, 4095, 4096, 4097, 16383, 16385, 65535, 65536, 65537, 131071, 131073,
+             3 * 65536 + 4099]
     specs = workloads.custom_layout(sizes)
     r = Run(specs, 12)
     for _ in range(4):
@@ -109,6 +110,25 @@ def test_edge_sizes_and_misaligned_views():
         assert (m[i].cpu().numpy() == rs.m).all() and (v[i].cpu().numpy() == rs.v).all()
         assert (p[i].cpu().numpy().view(np.uint32) == rs.p.view(np.uint32)).all()
         assert float(opt.amax_m[i]) == float(rs.amax_m[0]) and float(opt.scale_v[i]) == float(rs.scale_v[0])
+
+
+@pytest.mark.parametrize("chunk", [4096, 16384, 131072])
+def test_results_do_not_depend_on_the_chunk_length(chunk):
+    specs = workloads.custom_layout([300001, 4096, 17, 131072 * 2 + 3])
+    runs = []
+    for ce in (0, chunk):
+        M = workloads.FlatModel(specs, torch.device("cuda:0"))
+        workloads.init_params_into(specs, M.views(M.p), 19)
+        opt = FP8AdamW(M.views(M.p), M.views(M.g), m=M.views(M.m), v=M.views(M.v), scale_m=M.scale_m,
+                       scale_v=M.scale_v, amax_m=M.amax_m, amax_v=M.amax_v, chunk_elems=ce)
+        sig = workloads.tensor_sigmas(specs, 19)
+        for t in range(1, 5):
+            workloads.grads_into(specs, M.views(M.g), 19, t, sig)
+            opt.step()
+        torch.cuda.synchronize()
+        runs.append(M)
+    for name in ("p", "m", "v", "scale_m", "scale_v", "amax_m", "amax_v"):
+        assert torch.equal(getattr(runs[0], name).view(torch.uint8), getattr(runs[1], name).view(torch.uint8)), name
 
 
 def test_zero_gradients_keep_scale_and_decay_params():

@@ -1,12 +1,9 @@
 """Multi-rank host logic with world_size 2 on the gloo backend (CPU)."""
 import io
-import json
 import os
 import socket
-import sys
 from contextlib import redirect_stdout
 
-import pytest
 import torch.multiprocessing as mp
 
 from fp8_quantized_adam_b200 import ranks, workloads
