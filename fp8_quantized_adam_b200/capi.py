@@ -19,6 +19,7 @@ ERR_CUDA = -3
 ERR_OOM = -4
 ERR_WRONG_DEVICE = -5
 ERR_NOALLOC_LIMIT = -6
+ERR_DEVICE_TIMEOUT = -7
 NOALLOC_MAX_TENSORS = 4096
 
 E4M3, E5M2, FP32 = 0, 1, 2
@@ -26,6 +27,7 @@ FLAG_STATS = 1
 FLAG_JIT_EVERY_STEP = 2
 FLAG_UPDATE_FROM_STORED = 4
 FLAG_STOCHASTIC_ROUNDING = 8
+FLAG_NO_TMA = 16
 
 
 class fp8adam_tensor(ctypes.Structure):
@@ -91,6 +93,8 @@ def lib() -> ctypes.CDLL:
                                         ctypes.POINTER(vp)]
         L.fp8adam_step_ex.restype = ctypes.c_int
         L.fp8adam_step_ex.argtypes = [vp, ctypes.POINTER(fp8adam_step_params), vp]
+        L.fp8adam_check.restype = ctypes.c_int
+        L.fp8adam_check.argtypes = [vp, vp]
         L.fp8adam_get_grad_info.restype = ctypes.c_int
         L.fp8adam_get_grad_info.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint32), vp]
         L.fp8adam_step_noalloc.restype = ctypes.c_int
@@ -153,6 +157,10 @@ def fp8adam_reset_stats(ctx: int, cuda_stream: int) -> None:
     _check("fp8adam_reset_stats", lib().fp8adam_reset_stats(ctx, cuda_stream))
 
 
+def fp8adam_check(ctx: int, cuda_stream: int) -> None:
+    _check("fp8adam_check", lib().fp8adam_check(ctx, cuda_stream))
+
+
 def fp8adam_destroy(ctx: int) -> None:
     _check("fp8adam_destroy", lib().fp8adam_destroy(ctx))
 
@@ -186,4 +194,4 @@ def fp8adam_step_noalloc(tensors, num_tensors: int, scale_m: int, scale_v: int, 
 EXPORTED = ["fp8adam_create", "fp8adam_step", "fp8adam_get_stats", "fp8adam_reset_stats",
             "fp8adam_destroy", "fp8adam_strerror", "fp8adam_encode", "fp8adam_encode_bits_range",
             "fp8adam_decode", "fp8adam_launch_count", "fp8adam_step_noalloc", "fp8adam_create_ex",
-            "fp8adam_step_ex", "fp8adam_get_grad_info"]
+            "fp8adam_step_ex", "fp8adam_get_grad_info", "fp8adam_check"]

@@ -19,6 +19,7 @@
 #include "fp8_codec.cuh"
 #include "fp8adam_ext.cuh"
 #include "fp8adam_step.cuh"
+#include "fp8adam_step_tma.cuh"
 
 using namespace fp8adam;
 
@@ -127,6 +128,15 @@ StepFn pick_amax(int mf, int vf) {
   return t[mf][vf];
 }
 
+using TmaFn = void (*)(const StepArgs, uint32_t*);
+template <int MF, int VF, bool S> TmaFn tma_fn() { return &fp8adam_step_tma_kernel<MF, VF, S>; }
+TmaFn pick_tma(int mf, int vf, bool stats) {  // FP8 formats only
+  static const TmaFn t[2][2][2] = {
+      {{tma_fn<0, 0, false>(), tma_fn<0, 0, true>()}, {tma_fn<0, 1, false>(), tma_fn<0, 1, true>()}},
+      {{tma_fn<1, 0, false>(), tma_fn<1, 0, true>()}, {tma_fn<1, 1, false>(), tma_fn<1, 1, true>()}}};
+  return t[mf][vf][stats ? 1 : 0];
+}
+
 using ExtFn = void (*)(const ExtArgs);
 template <int MF, int VF, bool S> ExtFn ext_fn() { return &fp8adam_step_ext_kernel<MF, VF, S>; }
 template <int MF, int VF> ExtFn aext_fn() { return &fp8adam_amax_ext_kernel<MF, VF>; }
@@ -169,6 +179,8 @@ struct fp8adam_ctx {
   uint64_t seed = 0;
   uint16_t** d_bf16 = nullptr;  // device [T] bf16 outputs, or null
   bool ext = false;             // any option on: the variant kernels run
+  bool tma = false;             // default step through the TMA-staged kernel
+  uint32_t* d_error = nullptr;  // device error word (bounded waits that ran out)
   // gradient pre-pass of fp8adam_step_ex: [chunks] partials, non-finite
   // count, multiplier, skip flag, norm
   double* d_partial = nullptr;
@@ -184,6 +196,7 @@ static void free_ctx(fp8adam_ctx* c) {
   if (!c) return;
   cudaFree(c->d_tensors);
   cudaFree(c->d_chunks);
+  cudaFree(c->d_error);
   cudaFree(c->d_bf16);
   cudaFree(c->d_partial);
   cudaFree(c->d_nonfinite);
@@ -200,7 +213,8 @@ extern "C" int fp8adam_create(const fp8adam_tensor* tensors, int32_t num_tensors
                               int32_t v_fmt, uint32_t flags, fp8adam_ctx** out) {
   if (!out) return FP8ADAM_ERR_INVALID_ARG;
   *out = nullptr;
-  if (flags & ~(FP8ADAM_FLAG_STATS | FP8ADAM_FLAG_JIT_EVERY_STEP)) return FP8ADAM_ERR_INVALID_ARG;
+  if (flags & ~(FP8ADAM_FLAG_STATS | FP8ADAM_FLAG_JIT_EVERY_STEP | FP8ADAM_FLAG_NO_TMA))
+    return FP8ADAM_ERR_INVALID_ARG;
   fp8adam_options o;
   std::memset(&o, 0, sizeof(o));
   o.scale_m = scale_m;
@@ -225,7 +239,7 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
     return FP8ADAM_ERR_INVALID_ARG;
   if (m_fmt < 0 || m_fmt > 2 || v_fmt < 0 || v_fmt > 2) return FP8ADAM_ERR_UNSUPPORTED_FMT;
   if (flags & ~(FP8ADAM_FLAG_STATS | FP8ADAM_FLAG_JIT_EVERY_STEP | FP8ADAM_FLAG_UPDATE_FROM_STORED |
-                FP8ADAM_FLAG_STOCHASTIC_ROUNDING))
+                FP8ADAM_FLAG_STOCHASTIC_ROUNDING | FP8ADAM_FLAG_NO_TMA))
     return FP8ADAM_ERR_INVALID_ARG;
   if (opts->chunk_elems < 0 || opts->chunk_elems > kChunk || opts->chunk_elems % kTile != 0)
     return FP8ADAM_ERR_INVALID_ARG;
@@ -323,12 +337,21 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
       cudaMalloc(&c->d_grad_mult, sizeof(float)) != cudaSuccess ||
       cudaMalloc(&c->d_skip, sizeof(uint32_t)) != cudaSuccess ||
       cudaMalloc(&c->d_norm, sizeof(double)) != cudaSuccess ||
+      cudaMalloc(&c->d_error, sizeof(uint32_t)) != cudaSuccess ||
       (opts->param_bf16 && cudaMalloc(&c->d_bf16, T * sizeof(uint16_t*)) != cudaSuccess)) {
     cudaGetLastError();
     free_ctx(c);
     return FP8ADAM_ERR_OOM;
   }
+  c->tma = m_fmt != FP8ADAM_FP32 && v_fmt != FP8ADAM_FP32 && !(flags & FP8ADAM_FLAG_NO_TMA);
+  if (c->tma && cudaFuncSetAttribute((const void*)pick_tma(m_fmt, v_fmt, (flags & FP8ADAM_FLAG_STATS) != 0),
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmemBytes) != cudaSuccess) {
+    cudaGetLastError();
+    free_ctx(c);
+    return FP8ADAM_ERR_CUDA;
+  }
   if (cudaMemset(c->d_skip, 0, sizeof(uint32_t)) != cudaSuccess ||
+      cudaMemset(c->d_error, 0, sizeof(uint32_t)) != cudaSuccess ||
       cudaMemset(c->d_norm, 0, sizeof(double)) != cudaSuccess ||
       (opts->param_bf16 &&
        cudaMemcpy(c->d_bf16, opts->param_bf16, T * sizeof(uint16_t*), cudaMemcpyHostToDevice) != cudaSuccess) ||
@@ -403,7 +426,10 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
       a.amax_in_m = reinterpret_cast<const uint32_t*>(ctx->amax_m);
       a.amax_in_v = reinterpret_cast<const uint32_t*>(ctx->amax_v);
     }
-    pick_step(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(a);
+    if (ctx->tma)
+      pick_tma(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, kTmaSmemBytes, st>>>(a, ctx->d_error);
+    else
+      pick_step(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(a);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return last_error();
   }
@@ -517,6 +543,16 @@ extern "C" int fp8adam_reset_stats(fp8adam_ctx* ctx, void* cuda_stream) {
              : FP8ADAM_ERR_CUDA;
 }
 
+extern "C" int fp8adam_check(fp8adam_ctx* ctx, void* cuda_stream) {
+  if (!ctx) return FP8ADAM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  uint32_t e = 0;
+  if (cudaMemcpyAsync(&e, ctx->d_error, sizeof(e), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return FP8ADAM_ERR_CUDA;
+  return e ? FP8ADAM_ERR_DEVICE_TIMEOUT : FP8ADAM_OK;
+}
+
 extern "C" int fp8adam_destroy(fp8adam_ctx* ctx) {
   if (!ctx) return FP8ADAM_OK;
   const int rc = cudaDeviceSynchronize() == cudaSuccess ? FP8ADAM_OK : FP8ADAM_ERR_CUDA;
@@ -533,6 +569,7 @@ extern "C" const char* fp8adam_strerror(int code) {
     case FP8ADAM_ERR_OOM: return "device allocation failed";
     case FP8ADAM_ERR_WRONG_DEVICE: return "current device differs from the context's";
     case FP8ADAM_ERR_NOALLOC_LIMIT: return "more tensors than the allocation-free step holds (FP8ADAM_NOALLOC_MAX_TENSORS)";
+    case FP8ADAM_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait for its copies ran out; the state is not usable";
     default: return "unknown error";
   }
 }

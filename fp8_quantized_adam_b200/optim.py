@@ -47,7 +47,8 @@ class FP8AdamW:
                  jit_every_step: bool = False, margin_m: int = 0, margin_v: int = 0,
                  amax_history_len: int = 0, update_from_stored: bool = False,
                  stochastic_rounding: bool = False, seed: int = 0,
-                 param_bf16: Optional[List[torch.Tensor]] = None, chunk_elems: int = 0):
+                 param_bf16: Optional[List[torch.Tensor]] = None, chunk_elems: int = 0,
+                 tma: bool = True):
         if len(params) == 0 or len(params) != len(grads):
             raise ValueError("need matching, non-empty param and grad lists")
         self.params, self.grads = list(params), list(grads)
@@ -81,7 +82,8 @@ class FP8AdamW:
             arr[i] = capi.fp8adam_tensor(p.data_ptr(), g.data_ptr(), mm.data_ptr(), vv.data_ptr(), p.numel())
         flags = ((capi.FLAG_STATS if stats else 0) | (capi.FLAG_JIT_EVERY_STEP if jit_every_step else 0)
                  | (capi.FLAG_UPDATE_FROM_STORED if update_from_stored else 0)
-                 | (capi.FLAG_STOCHASTIC_ROUNDING if stochastic_rounding else 0))
+                 | (capi.FLAG_STOCHASTIC_ROUNDING if stochastic_rounding else 0)
+                 | (0 if tma else capi.FLAG_NO_TMA))
         self.amax_history_len = int(amax_history_len)
         self.hist_m = self.hist_v = None
         if self.amax_history_len > 1:
@@ -126,6 +128,11 @@ class FP8AdamW:
         pre-pass (synchronises the stream)."""
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         return capi.fp8adam_get_grad_info(self.ctx, s.cuda_stream)
+
+    def check(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """Raise if a kernel's bounded wait ran out (synchronises the stream)."""
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        capi.fp8adam_check(self.ctx, s.cuda_stream)
 
     def stats(self, stream: Optional[torch.cuda.Stream] = None):
         s = stream if stream is not None else torch.cuda.current_stream(self.device)

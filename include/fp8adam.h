@@ -66,6 +66,7 @@ extern "C" {
 #define FP8ADAM_ERR_OOM (-4)             /* device allocation failed in create */
 #define FP8ADAM_ERR_WRONG_DEVICE (-5)    /* current device differs from create's */
 #define FP8ADAM_ERR_NOALLOC_LIMIT (-6)   /* more tensors than fp8adam_step_noalloc holds */
+#define FP8ADAM_ERR_DEVICE_TIMEOUT (-7)  /* a kernel's bounded wait ran out (see fp8adam_check) */
 
 /* Storage format of a moment. */
 typedef enum {
@@ -77,6 +78,11 @@ typedef enum {
 /* Flags of fp8adam_create. */
 #define FP8ADAM_FLAG_STATS 1u            /* count flushed v and saturated codes */
 #define FP8ADAM_FLAG_JIT_EVERY_STEP 2u   /* "current" scaling: pre-pass every step */
+#define FP8ADAM_FLAG_NO_TMA 16u          /* load through per-thread vector loads only
+                                            (for comparison; same results).  By
+                                            default, FP8 m and v on 16-byte
+                                            aligned tensors are staged through
+                                            shared memory with TMA bulk copies. */
 
 /* One tensor.  param: fp32[numel]; grad: bf16[numel] (raw bits); m, v:
  * uint8[numel] codes or fp32[numel] in FP8ADAM_FP32 mode.  Any numel >= 0
@@ -123,6 +129,12 @@ int fp8adam_get_stats(fp8adam_ctx* ctx, uint64_t* out, void* cuda_stream);
 
 /* Zeroes the counters (queued on cuda_stream). */
 int fp8adam_reset_stats(fp8adam_ctx* ctx, void* cuda_stream);
+
+/* Checks the context's device error word (waits for cuda_stream): returns
+ * FP8ADAM_OK, or FP8ADAM_ERR_DEVICE_TIMEOUT if a step kernel's bounded wait
+ * for its shared-memory copies ran out (a chunk was then left unfinished and
+ * the state is not usable).  Host-side only otherwise. */
+int fp8adam_check(fp8adam_ctx* ctx, void* cuda_stream);
 
 /* Frees the context (synchronises the device first).  NULL is accepted. */
 int fp8adam_destroy(fp8adam_ctx* ctx);

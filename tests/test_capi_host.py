@@ -98,3 +98,5 @@ def test_option_entry_points_reject_bad_arguments_on_host(L):
     sp = capi.fp8adam_step_params(1e-3, 0.9, 0.95, 1e-8, 0.1, 1, 1.0, 0.0, 0)
     assert L.fp8adam_step_ex(None, ctypes.byref(sp), None) == capi.ERR_INVALID_ARG
     assert L.fp8adam_get_grad_info(None, None, None, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_check(None, None) == capi.ERR_INVALID_ARG
+    assert "not usable" in capi.fp8adam_strerror(capi.ERR_DEVICE_TIMEOUT)

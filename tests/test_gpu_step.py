@@ -131,6 +131,30 @@ def test_results_do_not_depend_on_the_chunk_length(chunk):
         assert torch.equal(getattr(runs[0], name).view(torch.uint8), getattr(runs[1], name).view(torch.uint8)), name
 
 
+@pytest.mark.parametrize("fmts", [(E4, E5), (E4, E4), (E5, E4), (E5, E5)], ids=["m4v5", "m4v4", "m5v4", "m5v5"])
+def test_tma_staged_and_vector_paths_agree(fmts):
+    """The shared-memory (TMA bulk copy) path and the per-thread vector path
+    give identical state, counters included, on ragged sizes; the device
+    error word stays clear."""
+    specs = workloads.custom_layout([300001, 4096, 17, 131072 * 2 + 2049, 2048, 2047, 6144 + 16])
+    runs = []
+    for tma in (True, False):
+        M = workloads.FlatModel(specs, torch.device("cuda:0"))
+        workloads.init_params_into(specs, M.views(M.p), 23)
+        opt = FP8AdamW(M.views(M.p), M.views(M.g), m_fmt=fmts[0], v_fmt=fmts[1], m=M.views(M.m), v=M.views(M.v),
+                       scale_m=M.scale_m, scale_v=M.scale_v, amax_m=M.amax_m, amax_v=M.amax_v, stats=True,
+                       tma=tma, chunk_elems=16384)
+        sig = workloads.tensor_sigmas(specs, 23)
+        for t in range(1, 6):
+            workloads.grads_into(specs, M.views(M.g), 23, t, sig)
+            opt.step()
+        opt.check()
+        runs.append((M, opt.stats()))
+    for name in ("p", "m", "v", "scale_m", "scale_v", "amax_m", "amax_v"):
+        assert torch.equal(getattr(runs[0][0], name).view(torch.uint8), getattr(runs[1][0], name).view(torch.uint8)), name
+    assert runs[0][1] == runs[1][1]
+
+
 def test_zero_gradients_keep_scale_and_decay_params():
     specs = workloads.custom_layout([5000])
     r = Run(specs, 14)
