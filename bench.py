@@ -192,14 +192,14 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(name: str, n: int) -> dict:
+def workload_config(name: str, n: int, variant: str = "default") -> dict:
     from fp8_quantized_adam_b200 import workloads
 
     specs = workloads.layout(name)
     return {"workload": name, "params_per_gpu": workloads.total_params(specs), "tensors": len(specs),
             "m_fmt": "e4m3", "v_fmt": "e5m2", "grads": "bf16, per-tensor N(0, 10^U(-5,-2)), 0.1% x100",
             "l2": "inputs larger than L2 (94.3 GB of traffic per step vs 126 MB L2), no flush",
-            "parallelism": "independent shard per GPU x%d" % n,
+            "parallelism": "independent shard per GPU x%d" % n, "variant": variant,
             "hparams": {"lr": 3e-4, "beta1": 0.9, "beta2": 0.95, "eps": 1e-8, "weight_decay": 0.1}}
 
 
@@ -228,13 +228,20 @@ def our_arm(args):
     workloads.init_params_into(specs, model.views(model.p), seed)
     sig = workloads.tensor_sigmas(specs, cfg)
     workloads.grads_into(specs, model.views(model.g), seed, 1, sig)
+    opt_kw, step_kw = {}, {}
+    if args.variant == "sr":
+        opt_kw = dict(stochastic_rounding=True, seed=1234)
+    elif args.variant == "history":
+        opt_kw = dict(amax_history_len=16)
+    elif args.variant == "clip":
+        step_kw = dict(loss_scale=1024.0, max_norm=1.0, skip_nonfinite=True)
     opt = FP8AdamW(model.views(model.p), model.views(model.g), m=model.views(model.m), v=model.views(model.v),
                    scale_m=model.scale_m, scale_v=model.scale_v, amax_m=model.amax_m, amax_v=model.amax_v,
-                   chunk_elems=args.chunk_elems, tma=not args.no_tma)
+                   chunk_elems=args.chunk_elems, tma=not args.no_tma, **opt_kw)
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
-        opt.step()
+        opt.step(**step_kw)
     barrier()
 
     # ---- device-timed region: K steps, inputs resident
@@ -249,7 +256,7 @@ def our_arm(args):
     t_start.record(stream)
     for k in range(args.steps):
         ev[k][0].record(stream)
-        opt.step()
+        opt.step(**step_kw)
         ev[k][1].record(stream)
     t_end.record(stream)
     barrier()
@@ -278,7 +285,7 @@ def our_arm(args):
             e0.record(stream)
             for _ in range(e2e_steps):
                 model.g.copy_(g_host, non_blocking=True)
-                opt.step()
+                opt.step(**step_kw)
                 am_host[:len(specs)].copy_(model.amax_m, non_blocking=True)
                 am_host[len(specs):].copy_(model.amax_v, non_blocking=True)
             e1.record(stream)
@@ -293,15 +300,20 @@ def our_arm(args):
 
     peak, peak_kind = hbm_peak()
     avg_kernel_s = sum(kernel_ms) / len(kernel_ms) / 1e3
-    achieved = BYTES_PER_PARAM * n_params / avg_kernel_s / 1e9
+    # bytes per param of one step: the fused clip/skip variant reads the
+    # gradients once more in its norm pre-pass
+    bpp = BYTES_PER_PARAM + (2 if args.variant == "clip" else 0)
+    achieved = bpp * n_params / avg_kernel_s / 1e9
     traffic = None
-    if TRAFFIC_PER_PARAM is not None and KERNEL_SHA == kernel_sha():
+    if TRAFFIC_PER_PARAM is not None and KERNEL_SHA == kernel_sha() and args.variant == "default" and not args.no_tma:
         traffic = TRAFFIC_PER_PARAM * n_params
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else peak_kind,
                 "traffic": traffic,
-                "kernel": "fp8adam_step_kernel<E4M3,E5M2>" if args.no_tma else "fp8adam_step_tma_kernel<E4M3,E5M2>",
-                "algorithmic_bytes_per_launch": BYTES_PER_PARAM * n_params,
+                "kernel": ("fp8adam_step_ext_kernel<E4M3,E5M2>" + (" + grad-norm pre-pass" if args.variant == "clip" else "")
+                           if args.variant != "default" else
+                           "fp8adam_step_kernel<E4M3,E5M2>" if args.no_tma else "fp8adam_step_tma_kernel<E4M3,E5M2>"),
+                "algorithmic_bytes_per_launch": bpp * n_params,
                 "kernel_ms_avg": avg_kernel_s * 1e3, "kernel_ms_min": min(kernel_ms),
                 "kernel_ms_p50": sorted(kernel_ms)[len(kernel_ms) // 2],
                 "kernel_ms_p90": sorted(kernel_ms)[min(len(kernel_ms) - 1, (9 * len(kernel_ms)) // 10)],
@@ -321,9 +333,9 @@ def our_arm(args):
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": elapsed * 1e3 / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": workload_config(name, world), "roofline": roofline, "cpu_baseline": cpu,
+                "config": workload_config(name, world, args.variant), "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": e2e, "gpu_launches": launches, "clocks": clk,
-                "gb_per_s": world * BYTES_PER_PARAM * n_params * args.steps / elapsed / 1e9}
+                "gb_per_s": world * bpp * n_params * args.steps / elapsed / 1e9}
         print(json.dumps(line), flush=True)
     ranks.finish()
 
@@ -403,6 +415,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--chunk-elems", type=int, default=0, help="elements per CTA (0: chosen by the library)")
     ap.add_argument("--no-tma", action="store_true", help="per-thread vector loads instead of TMA staging")
+    ap.add_argument("--variant", choices=["default", "sr", "history", "clip"], default="default",
+                    help="step options: stochastic rounding, amax history 16, fused loss-scale/clip/skip")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--report", choices=["ablation"], default=None,
