@@ -192,6 +192,15 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
+def kernel_name(args) -> str:
+    """The step kernel a run times (plus the norm pre-pass for clipping)."""
+    if args.variant == "default":
+        return "fp8adam_step_kernel<E4M3,E5M2>" if args.no_tma else "fp8adam_step_tma_kernel<E4M3,E5M2>"
+    base = ("fp8adam_step_ext_kernel<E4M3,E5M2>" if args.no_tma else
+            "fp8adam_step_ext_tma_kernel<E4M3,E5M2,SR=%d>" % (args.variant == "sr"))
+    return base + (" + grad-norm pre-pass" if args.variant == "clip" else "")
+
+
 def workload_config(name: str, n: int, variant: str = "default") -> dict:
     from fp8_quantized_adam_b200 import workloads
 
@@ -310,9 +319,7 @@ def our_arm(args):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else peak_kind,
                 "traffic": traffic,
-                "kernel": ("fp8adam_step_ext_kernel<E4M3,E5M2>" + (" + grad-norm pre-pass" if args.variant == "clip" else "")
-                           if args.variant != "default" else
-                           "fp8adam_step_kernel<E4M3,E5M2>" if args.no_tma else "fp8adam_step_tma_kernel<E4M3,E5M2>"),
+                "kernel": kernel_name(args),
                 "algorithmic_bytes_per_launch": bpp * n_params,
                 "kernel_ms_avg": avg_kernel_s * 1e3, "kernel_ms_min": min(kernel_ms),
                 "kernel_ms_p50": sorted(kernel_ms)[len(kernel_ms) // 2],

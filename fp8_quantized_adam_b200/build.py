@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfp8adam.so")
 SOURCES = [os.path.join(CSRC, "fp8adam_capi.cu"), os.path.join(CSRC, "fp8adam_noalloc.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fp8_codec.cuh", "fp8adam_step.cuh", "fp8adam_ext.cuh", "fp8adam_step_tma.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fp8_codec.cuh", "fp8adam_step.cuh", "fp8adam_ext.cuh", "fp8adam_step_tma.cuh", "fp8adam_ext_tma.cuh")] + [
     os.path.join(ROOT, "include", "fp8adam.h")]
 
 NVCC_FLAGS = [

@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.fp8adam_encode_bits_range.argtypes = [i32, u32, i64, vp, i32, vp]
         L.fp8adam_decode.restype = ctypes.c_int
         L.fp8adam_decode.argtypes = [i32, vp, vp, i64, i32, vp]
+        L.fp8adam_encode_sr.restype = ctypes.c_int
+        L.fp8adam_encode_sr.argtypes = [i32, vp, vp, vp, i64, vp]
         L.fp8adam_launch_count.restype = ctypes.c_uint64
         L.fp8adam_launch_count.argtypes = []
         L.fp8adam_create_ex.restype = ctypes.c_int
@@ -173,6 +175,10 @@ def fp8adam_encode_bits_range(fmt: int, first: int, n: int, out: int, impl: int,
     _check("fp8adam_encode_bits_range", lib().fp8adam_encode_bits_range(fmt, first, n, out, impl, cuda_stream))
 
 
+def fp8adam_encode_sr(fmt: int, x: int, r: int, out: int, n: int, cuda_stream: int) -> None:
+    _check("fp8adam_encode_sr", lib().fp8adam_encode_sr(fmt, x, r, out, n, cuda_stream))
+
+
 def fp8adam_decode(fmt: int, codes: int, out: int, n: int, impl: int, cuda_stream: int) -> None:
     _check("fp8adam_decode", lib().fp8adam_decode(fmt, codes, out, n, impl, cuda_stream))
 
@@ -194,4 +200,4 @@ def fp8adam_step_noalloc(tensors, num_tensors: int, scale_m: int, scale_v: int, 
 EXPORTED = ["fp8adam_create", "fp8adam_step", "fp8adam_get_stats", "fp8adam_reset_stats",
             "fp8adam_destroy", "fp8adam_strerror", "fp8adam_encode", "fp8adam_encode_bits_range",
             "fp8adam_decode", "fp8adam_launch_count", "fp8adam_step_noalloc", "fp8adam_create_ex",
-            "fp8adam_step_ex", "fp8adam_get_grad_info", "fp8adam_check"]
+            "fp8adam_step_ex", "fp8adam_get_grad_info", "fp8adam_check", "fp8adam_encode_sr"]

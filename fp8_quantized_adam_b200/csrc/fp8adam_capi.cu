@@ -18,6 +18,7 @@
 #include "../../include/fp8adam.h"
 #include "fp8_codec.cuh"
 #include "fp8adam_ext.cuh"
+#include "fp8adam_ext_tma.cuh"
 #include "fp8adam_step.cuh"
 #include "fp8adam_step_tma.cuh"
 
@@ -96,6 +97,14 @@ __global__ void decode_kernel(const uint8_t* __restrict__ c, float* __restrict__
   }
 }
 
+template <int FMT>
+__global__ void encode_sr_kernel(const float* __restrict__ x, const uint32_t* __restrict__ r,
+                                 uint8_t* __restrict__ out, int64_t n) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+    out[i] = (uint8_t)enc1_sr<FMT>(x[i], r[i]);
+}
+
 int grid_for(int64_t n, int per_thread) {
   const int64_t want = (n + (int64_t)256 * per_thread - 1) / ((int64_t)256 * per_thread);
   const int64_t cap = 148 * 16;
@@ -150,6 +159,20 @@ ExtFn pick_ext(int mf, int vf, bool stats) {
       {{ext_fn<2, 0, false>(), ext_fn<2, 0, true>()}, {ext_fn<2, 1, false>(), ext_fn<2, 1, true>()},
        {ext_fn<2, 2, false>(), ext_fn<2, 2, true>()}}};
   return t[mf][vf][stats ? 1 : 0];
+}
+using ExtTmaFn = void (*)(const ExtArgs, uint32_t*);
+template <int MF, int VF, bool S, bool SR> ExtTmaFn ext_tma_fn() { return &fp8adam_step_ext_tma_kernel<MF, VF, S, SR>; }
+ExtTmaFn pick_ext_tma(int mf, int vf, bool stats, bool sr) {  // FP8 formats only
+  static const ExtTmaFn t[2][2][2][2] = {
+      {{{ext_tma_fn<0, 0, false, false>(), ext_tma_fn<0, 0, false, true>()},
+        {ext_tma_fn<0, 0, true, false>(), ext_tma_fn<0, 0, true, true>()}},
+       {{ext_tma_fn<0, 1, false, false>(), ext_tma_fn<0, 1, false, true>()},
+        {ext_tma_fn<0, 1, true, false>(), ext_tma_fn<0, 1, true, true>()}}},
+      {{{ext_tma_fn<1, 0, false, false>(), ext_tma_fn<1, 0, false, true>()},
+        {ext_tma_fn<1, 0, true, false>(), ext_tma_fn<1, 0, true, true>()}},
+       {{ext_tma_fn<1, 1, false, false>(), ext_tma_fn<1, 1, false, true>()},
+        {ext_tma_fn<1, 1, true, false>(), ext_tma_fn<1, 1, true, true>()}}}};
+  return t[mf][vf][stats ? 1 : 0][sr ? 1 : 0];
 }
 ExtFn pick_amax_ext(int mf, int vf) {
   static const ExtFn t[3][3] = {{aext_fn<0, 0>(), aext_fn<0, 1>(), aext_fn<0, 2>()},
@@ -344,8 +367,12 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
     return FP8ADAM_ERR_OOM;
   }
   c->tma = m_fmt != FP8ADAM_FP32 && v_fmt != FP8ADAM_FP32 && !(flags & FP8ADAM_FLAG_NO_TMA);
-  if (c->tma && cudaFuncSetAttribute((const void*)pick_tma(m_fmt, v_fmt, (flags & FP8ADAM_FLAG_STATS) != 0),
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmemBytes) != cudaSuccess) {
+  const bool stats_on = (flags & FP8ADAM_FLAG_STATS) != 0;
+  const bool sr_on = (flags & FP8ADAM_FLAG_STOCHASTIC_ROUNDING) != 0;
+  if (c->tma && (cudaFuncSetAttribute((const void*)pick_tma(m_fmt, v_fmt, stats_on),
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmemBytes) != cudaSuccess ||
+                 cudaFuncSetAttribute((const void*)pick_ext_tma(m_fmt, v_fmt, stats_on, sr_on),
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmemBytes) != cudaSuccess)) {
     cudaGetLastError();
     free_ctx(c);
     return FP8ADAM_ERR_CUDA;
@@ -477,7 +504,11 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
     a.amax_in_v = reinterpret_cast<const uint32_t*>(ctx->amax_v);
   }
   e.s = a;
-  pick_ext(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(e);
+  if (ctx->tma)
+    pick_ext_tma(ctx->m_fmt, ctx->v_fmt, stats, (e.flags & FP8ADAM_FLAG_STOCHASTIC_ROUNDING) != 0)
+        <<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
+  else
+    pick_ext(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return last_error();
 }
@@ -603,6 +634,18 @@ extern "C" int fp8adam_encode_bits_range(int32_t fmt, uint32_t first, int64_t n,
   if (n == 0) return FP8ADAM_OK;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   FP8ADAM_CODEC_DISPATCH(encode_bits_kernel, grid_for(n, 4), first, out, n);
+  return last_error();
+}
+
+extern "C" int fp8adam_encode_sr(int32_t fmt, const float* x, const uint32_t* r, uint8_t* out, int64_t n,
+                                 void* cuda_stream) {
+  if (fmt < 0 || fmt > 1) return FP8ADAM_ERR_UNSUPPORTED_FMT;
+  if (n < 0 || (n > 0 && (!x || !r || !out))) return FP8ADAM_ERR_INVALID_ARG;
+  if (n == 0) return FP8ADAM_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (fmt == 0) encode_sr_kernel<0><<<grid_for(n, 1), 256, 0, st>>>(x, r, out, n);
+  else encode_sr_kernel<1><<<grid_for(n, 1), 256, 0, st>>>(x, r, out, n);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   return last_error();
 }
 

@@ -119,8 +119,18 @@ __device__ __forceinline__ float pow2scale_margin(float amax, float s_prev, int 
 }
 
 // ------------------------------------------------------------ encode/store
+// Rounding of the codes: fixed at compile time (the staged kernels, one
+// instantiation each) or read from ExtArgs::flags (the per-thread-load kernel).
+enum SrMode : int { kRoundNearest = 0, kRoundStochastic = 1, kRoundByFlag = 2 };
+
+template <int SRM>
+__device__ __forceinline__ bool use_sr(const ExtArgs& a) {
+  if constexpr (SRM == kRoundByFlag) return (a.flags & kExtStochastic) != 0;
+  else return SRM == kRoundStochastic;
+}
+
 // Encodes one moment value (x * s) and returns the value the update reads.
-template <int FMT, bool STATS, bool IS_V>
+template <int FMT, bool STATS, bool IS_V, int SRM>
 __device__ __forceinline__ float ext_q(const ExtArgs& a, float x, float s, float inv_s, uint32_t r, uint32_t& code,
                                        uint32_t& flushed, uint32_t& sat) {
   if constexpr (FMT == kFP32) {
@@ -128,7 +138,7 @@ __device__ __forceinline__ float ext_q(const ExtArgs& a, float x, float s, float
     return x;
   } else {
     const float y = __fmul_rn(x, s);
-    code = (a.flags & kExtStochastic) ? enc1_sr<FMT>(y, r) : enc1_hw<FMT>(y);
+    code = use_sr<SRM>(a) ? enc1_sr<FMT>(y, r) : enc1_hw<FMT>(y);
     if constexpr (STATS) {
       sat += fabsf(y) > FmtTraits<FMT>::kMax ? 1u : 0u;
       if constexpr (IS_V) flushed += (x > 0.0f && (code & 0x7Fu) == 0u) ? 1u : 0u;
@@ -144,12 +154,12 @@ struct ExtSeg {  // per tensor segment
 };
 
 // One element (tails, unaligned tensors).
-template <int MF, int VF, bool STATS>
+template <int MF, int VF, bool STATS, int SRM>
 __device__ __forceinline__ void ext_element(const ExtArgs& a, const TensorDesc& td, const ExtSeg& sg, int64_t i,
                                             float& am, float& av, uint32_t& flushed, uint32_t& sat) {
   const StepConsts& c = a.s.c;
   uint32_t rm = 0, rv = 0;
-  if (a.flags & kExtStochastic) {
+  if (use_sr<SRM>(a)) {
     const uint4 r = sr_words(a, sg.ti, i >> 1);
     rm = (i & 1) ? r.z : r.x;
     rv = (i & 1) ? r.w : r.y;
@@ -160,8 +170,8 @@ __device__ __forceinline__ void ext_element(const ExtArgs& a, const TensorDesc& 
   am = fmax_nan(am, fabsf(mn));
   av = fmax_nan(av, fabsf(vn));
   uint32_t qm, qv;
-  const float mu = ext_q<MF, STATS, false>(a, mn, sg.s_m_new, sg.inv_s_m_new, rm, qm, flushed, sat);
-  const float vu = ext_q<VF, STATS, true>(a, vn, sg.s_v_new, sg.inv_s_v_new, rv, qv, flushed, sat);
+  const float mu = ext_q<MF, STATS, false, SRM>(a, mn, sg.s_m_new, sg.inv_s_m_new, rm, qm, flushed, sat);
+  const float vu = ext_q<VF, STATS, true, SRM>(a, vn, sg.s_v_new, sg.inv_s_v_new, rv, qv, flushed, sat);
   if constexpr (MF == kFP32) static_cast<float*>(td.m)[i] = mn; else static_cast<uint8_t*>(td.m)[i] = (uint8_t)qm;
   if constexpr (VF == kFP32) static_cast<float*>(td.v)[i] = vn; else static_cast<uint8_t*>(td.v)[i] = (uint8_t)qv;
   const float pn = update(c, td.p[i], mu, vu);
@@ -170,7 +180,7 @@ __device__ __forceinline__ void ext_element(const ExtArgs& a, const TensorDesc& 
 }
 
 // 16 elements of an aligned tensor (vector loads/stores, as the default step).
-template <int MF, int VF, bool STATS>
+template <int MF, int VF, bool STATS, int SRM>
 __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& td, const ExtSeg& sg, int64_t i,
                                             float& am, float& av, uint32_t& flushed, uint32_t& sat) {
   const StepConsts& c = a.s.c;
@@ -193,7 +203,7 @@ __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& 
     const float g[4] = {__fmul_rn(bf16_lo(gw[2 * k]), sg.gm), __fmul_rn(bf16_hi(gw[2 * k]), sg.gm),
                         __fmul_rn(bf16_lo(gw[2 * k + 1]), sg.gm), __fmul_rn(bf16_hi(gw[2 * k + 1]), sg.gm)};
     uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
-    if (a.flags & kExtStochastic) {
+    if (use_sr<SRM>(a)) {
       r0 = sr_words(a, sg.ti, (i + 4 * k) >> 1);
       r1 = sr_words(a, sg.ti, ((i + 4 * k) >> 1) + 1);
     }
@@ -205,8 +215,8 @@ __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& 
       moments(c, g[j], mo[j], vo[j], mn[j], vn[j]);
       am = fmax_nan(am, fabsf(mn[j]));
       av = fmax_nan(av, fabsf(vn[j]));
-      mu[j] = ext_q<MF, STATS, false>(a, mn[j], sg.s_m_new, sg.inv_s_m_new, rmj[j], qm[j], flushed, sat);
-      vu[j] = ext_q<VF, STATS, true>(a, vn[j], sg.s_v_new, sg.inv_s_v_new, rvj[j], qv[j], flushed, sat);
+      mu[j] = ext_q<MF, STATS, false, SRM>(a, mn[j], sg.s_m_new, sg.inv_s_m_new, rmj[j], qm[j], flushed, sat);
+      vu[j] = ext_q<VF, STATS, true, SRM>(a, vn[j], sg.s_v_new, sg.inv_s_v_new, rvj[j], qv[j], flushed, sat);
     }
     float pk[4] = {pv[k].x, pv[k].y, pv[k].z, pv[k].w};
 #pragma unroll
@@ -232,11 +242,12 @@ __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& 
 }
 
 // ------------------------------------------------------------ the variant step
-template <int MF, int VF, bool STATS>
-__device__ __forceinline__ void run_ext_segment(const ExtArgs& a, int ti, int64_t e0, int64_t e1, uint32_t units,
-                                                float gm, uint32_t (*red)[kThreads / 32]) {
+// Per-chunk constants: this step's decode scales, the encode scales from the
+// amax (or the max of the amax history) with the margin, the multiplier and
+// the bf16 output of tensor ti.
+template <int MF, int VF>
+__device__ __forceinline__ ExtSeg ext_setup(const ExtArgs& a, int ti, float gm) {
   const StepArgs& S = a.s;
-  const TensorDesc td = S.tensors[ti];
   ExtSeg sg;
   sg.ti = ti;
   sg.gm = gm;
@@ -261,19 +272,35 @@ __device__ __forceinline__ void run_ext_segment(const ExtArgs& a, int ti, int64_
   sg.inv_s_v = __fdiv_rn(1.0f, s_v);
   sg.inv_s_m_new = __fdiv_rn(1.0f, sg.s_m_new);
   sg.inv_s_v_new = __fdiv_rn(1.0f, sg.s_v_new);
+  return sg;
+}
 
-  float am = 0.0f, av = 0.0f;
-  uint32_t flushed = 0, sat = 0;
+// The vector path needs the tensor's four buffers and its bf16 output (if
+// any) 16-byte aligned.
+__device__ __forceinline__ bool ext_vec_ok(const TensorDesc& td, const ExtSeg& sg) {
+  return td.aligned && (sg.pb == nullptr || ((uintptr_t)sg.pb & 15u) == 0);
+}
+
+// Elements [e0, e1) of the chunk through the per-thread paths.
+template <int MF, int VF, bool STATS, int SRM>
+__device__ __forceinline__ void ext_range(const ExtArgs& a, const TensorDesc& td, const ExtSeg& sg, int64_t e0,
+                                          int64_t e1, float& am, float& av, uint32_t& flushed, uint32_t& sat) {
   int64_t scalar_from = e0;
-  const bool vec = td.aligned && (sg.pb == nullptr || ((uintptr_t)sg.pb & 15u) == 0);
-  if (vec) {
+  if (ext_vec_ok(td, sg)) {
     for (int64_t i = e0 + (int64_t)threadIdx.x * kVec; i + kVec <= e1; i += kTile)
-      ext_group16<MF, VF, STATS>(a, td, sg, i, am, av, flushed, sat);
+      ext_group16<MF, VF, STATS, SRM>(a, td, sg, i, am, av, flushed, sat);
     scalar_from = e0 + (e1 - e0) / kVec * kVec;
   }
   for (int64_t i = scalar_from + threadIdx.x; i < e1; i += kThreads)
-    ext_element<MF, VF, STATS>(a, td, sg, i, am, av, flushed, sat);
+    ext_element<MF, VF, STATS, SRM>(a, td, sg, i, am, av, flushed, sat);
+}
 
+// Block reduction of the chunk's amax (and counters), then the publish of
+// the tensor's amax, history slot and scales by the CTA that finishes it.
+template <bool STATS>
+__device__ __forceinline__ void ext_flush(const ExtArgs& a, int ti, int32_t nunits, const ExtSeg& sg, float am,
+                                          float av, uint32_t flushed, uint32_t sat, uint32_t (*red)[kThreads / 32]) {
+  const StepArgs& S = a.s;
   const uint32_t bm = block_max(__float_as_uint(am), red[0]);
   const uint32_t bv = block_max(__float_as_uint(av), red[1]);
   uint32_t bf = 0, bs = 0;
@@ -289,8 +316,8 @@ __device__ __forceinline__ void run_ext_segment(const ExtArgs& a, int ti, int64_
       if (bs) atomicAdd(S.stats + 1, (unsigned long long)bs);
     }
     __threadfence();
-    const uint32_t prev = atomicAdd(S.done + ti, units);
-    if (prev + units == (uint32_t)td.nunits) {
+    const uint32_t prev = atomicAdd(S.done + ti, 1u);
+    if (prev + 1u == (uint32_t)nunits) {
       __threadfence();
       const uint32_t fm = atomicExch(S.acc_m + ti, 0u);
       const uint32_t fv = atomicExch(S.acc_v + ti, 0u);
@@ -307,53 +334,91 @@ __device__ __forceinline__ void run_ext_segment(const ExtArgs& a, int ti, int64_
   }
 }
 
+// The per-thread-load variant step (fp32 moments, or staging switched off);
+// the rounding mode comes from the flags.
 template <int MF, int VF, bool STATS>
 __global__ void __launch_bounds__(kThreads, 2)
 fp8adam_step_ext_kernel(const ExtArgs a) {
   __shared__ uint32_t red[4][kThreads / 32];
   if (a.skip && *a.skip) return;  // a non-finite gradient: the step is skipped
   const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
-  for_each_segment(a.s, [&](int ti, int64_t e0, int64_t e1, uint32_t units) {
-    run_ext_segment<MF, VF, STATS>(a, ti, e0, e1, units, gm, red);
-  });
+  const Chunk ch = a.s.chunks[blockIdx.x];
+  const int ti = ch.tensor;
+  const TensorDesc td = a.s.tensors[ti];
+  const ExtSeg sg = ext_setup<MF, VF>(a, ti, gm);
+  float am = 0.0f, av = 0.0f;
+  uint32_t flushed = 0, sat = 0;
+  ext_range<MF, VF, STATS, kRoundByFlag>(a, td, sg, ch.start, ch.start + ch.len, am, av, flushed, sat);
+  ext_flush<STATS>(a, ti, td.nunits, sg, am, av, flushed, sat, red);
 }
 
 // ------------------------------------------------------------ amax pre-pass
 // Step-1 / current-scaling pre-pass of the variant step: the same moments
 // (with the gradient multiplier), no stores; accumulates into s.acc_m/acc_v.
+// 16 elements per thread-iteration with vector loads on aligned tensors.
 template <int MF, int VF>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, StepOccupancy<MF, VF>::kMinBlocks)
 fp8adam_amax_ext_kernel(const ExtArgs a) {
   __shared__ uint32_t red[2][kThreads / 32];
   if (a.skip && *a.skip) return;
   const StepArgs& S = a.s;
   const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
-  for_each_segment(S, [&](int ti, int64_t e0, int64_t e1, uint32_t) {
-    const TensorDesc td = S.tensors[ti];
-    const float inv_s_m = __fdiv_rn(1.0f, S.scale_m[ti]);
-    const float inv_s_v = __fdiv_rn(1.0f, S.scale_v[ti]);
-    float am = 0.0f, av = 0.0f;
-    for (int64_t i = e0 + threadIdx.x; i < e1; i += kThreads) {
-      const float g = __fmul_rn(__uint_as_float((uint32_t)td.g[i] << 16), gm);
-      float mn, vn;
-      moments(S.c, g, load1<MF>(td.m, i, inv_s_m), load1<VF>(td.v, i, inv_s_v), mn, vn);
-      am = fmax_nan(am, fabsf(mn));
-      av = fmax_nan(av, fabsf(vn));
+  const Chunk ch = S.chunks[blockIdx.x];
+  const int ti = ch.tensor;
+  const TensorDesc td = S.tensors[ti];
+  const int64_t e0 = ch.start, e1 = ch.start + ch.len;
+  const float inv_s_m = __fdiv_rn(1.0f, S.scale_m[ti]);
+  const float inv_s_v = __fdiv_rn(1.0f, S.scale_v[ti]);
+  float am = 0.0f, av = 0.0f;
+  int64_t scalar_from = e0;
+  if (td.aligned) {
+    for (int64_t i = e0 + (int64_t)threadIdx.x * kVec; i + kVec <= e1; i += kTile) {
+      const uint4 g0 = ld_ro_u4(td.g + i);
+      const uint4 g1 = ld_ro_u4(td.g + i + 8);
+      Tile16<MF> tm;
+      Tile16<VF> tv;
+      tm.load(td.m, i);
+      tv.load(td.v, i);
+      const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float mo[4], vo[4];
+        tm.decode4(k, inv_s_m, mo);
+        tv.decode4(k, inv_s_v, vo);
+        const float g[4] = {__fmul_rn(bf16_lo(gw[2 * k]), gm), __fmul_rn(bf16_hi(gw[2 * k]), gm),
+                            __fmul_rn(bf16_lo(gw[2 * k + 1]), gm), __fmul_rn(bf16_hi(gw[2 * k + 1]), gm)};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float mn, vn;
+          moments(S.c, g[j], mo[j], vo[j], mn, vn);
+          am = fmax_nan(am, fabsf(mn));
+          av = fmax_nan(av, fabsf(vn));
+        }
+      }
     }
-    const uint32_t bm = block_max(__float_as_uint(am), red[0]);
-    const uint32_t bv = block_max(__float_as_uint(av), red[1]);
-    if (threadIdx.x == 0) {
-      if (bm) atomicMax(S.acc_m + ti, bm);
-      if (bv) atomicMax(S.acc_v + ti, bv);
-    }
-  });
+    scalar_from = e0 + (e1 - e0) / kVec * kVec;
+  }
+  for (int64_t i = scalar_from + threadIdx.x; i < e1; i += kThreads) {
+    const float g = __fmul_rn(__uint_as_float((uint32_t)td.g[i] << 16), gm);
+    float mn, vn;
+    moments(S.c, g, load1<MF>(td.m, i, inv_s_m), load1<VF>(td.v, i, inv_s_v), mn, vn);
+    am = fmax_nan(am, fabsf(mn));
+    av = fmax_nan(av, fabsf(vn));
+  }
+  const uint32_t bm = block_max(__float_as_uint(am), red[0]);
+  const uint32_t bv = block_max(__float_as_uint(av), red[1]);
+  if (threadIdx.x == 0) {
+    if (bm) atomicMax(S.acc_m + ti, bm);
+    if (bv) atomicMax(S.acc_v + ti, bv);
+  }
 }
 
 // ------------------------------------------------------------ grad-norm pre-pass
-// Per CTA: the sum of g^2 (each term exact in double) over its tiles, in a
-// fixed order (thread-sequential, then a fixed shuffle/shared-memory tree),
-// written to partial[blockIdx.x]; non-finite gradients are counted (not
-// summed).  The fixed grid makes the result reproducible run to run.
+// Per CTA: the sum of g^2 (each term exact in double) over its chunk, in a
+// fixed order (each thread's elements in sequence, then a fixed
+// shuffle/shared-memory tree), written to partial[blockIdx.x]; non-finite
+// gradients are counted (not summed).  The fixed grid makes the result
+// reproducible run to run.
 __device__ __forceinline__ double block_sum_d(double x, double* sm) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
@@ -368,24 +433,48 @@ __device__ __forceinline__ double block_sum_d(double x, double* sm) {
   return r;
 }
 
+// acc += g^2 for one bf16 gradient (bits b, low 16 bits).  A normal bf16 is
+// widened to double by placing its exponent and 7 mantissa bits (no
+// conversion instruction); g^2 has at most 16 significant bits, so the fused
+// multiply-add rounds once, exactly like adding the exact square.  Zero adds
+// nothing; inf and NaN are counted, not summed.
+__device__ __forceinline__ void sumsq1(uint32_t b, double& acc, uint32_t& bad) {
+  const uint32_t h = b & 0x7FFFu;
+  if (h - 0x80u < 0x7F00u) {  // exponent field 1..254
+    const double x = __hiloint2double((int)((h << 13) + (896u << 20)), 0);
+    acc = __fma_rn(x, x, acc);
+  } else if (h >= 0x7F80u) {
+    ++bad;
+  } else if (h != 0u) {  // subnormal
+    const double x = (double)__uint_as_float(h << 16);
+    acc = __fma_rn(x, x, acc);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads)
 fp8adam_gradnorm_partial_kernel(const StepArgs a, double* partial, unsigned long long* nonfinite) {
   __shared__ double red[kThreads / 32];
   __shared__ uint32_t redi[kThreads / 32];
   double acc = 0.0;
   uint32_t bad = 0;
-  for_each_segment(a, [&](int ti, int64_t e0, int64_t e1, uint32_t) {
-    const uint16_t* g = a.tensors[ti].g;
-    for (int64_t i = e0 + threadIdx.x; i < e1; i += kThreads) {
-      const uint32_t b = g[i];
-      if ((b & 0x7F80u) == 0x7F80u) {
-        ++bad;
-      } else {
-        const double x = (double)__uint_as_float(b << 16);
-        acc = __dadd_rn(acc, __dmul_rn(x, x));
+  const Chunk ch = a.chunks[blockIdx.x];
+  const TensorDesc td = a.tensors[ch.tensor];
+  const int64_t e0 = ch.start, e1 = ch.start + ch.len;
+  int64_t scalar_from = e0;
+  if (td.aligned) {
+    for (int64_t i = e0 + (int64_t)threadIdx.x * kVec; i + kVec <= e1; i += kTile) {
+      const uint4 g0 = ld_ro_u4(td.g + i);
+      const uint4 g1 = ld_ro_u4(td.g + i + 8);
+      const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        sumsq1(gw[k] & 0xFFFFu, acc, bad);
+        sumsq1(gw[k] >> 16, acc, bad);
       }
     }
-  });
+    scalar_from = e0 + (e1 - e0) / kVec * kVec;
+  }
+  for (int64_t i = scalar_from + threadIdx.x; i < e1; i += kThreads) sumsq1(td.g[i], acc, bad);
   const double s = block_sum_d(acc, red);
   const uint32_t nb = block_sum(bad, redi);
   if (threadIdx.x == 0) {

@@ -1,0 +1,142 @@
+// fp8adam_ext_tma.cuh -- the variant step (options of fp8adam_create_ex /
+// fp8adam_step_ex) with its loads staged through shared memory by bulk
+// copies, for FP8 m and v.
+//
+// The pipeline is the default staged step's (tma_stream: 3 x 16 KB stages,
+// one issuing thread, bounded waits, 4 CTAs of 256 threads per SM); the
+// element work adds the options to the default step's:
+//   - the gradient multiplier (loss-scale removal and clipping), one multiply;
+//   - the encode scales from the amax history and the margin (per chunk);
+//   - stochastic rounding (a compile-time switch: Philox4x32-10 words for two
+//     elements per call, and the integer SR encoder), or round-to-nearest
+//     with the hardware conversion;
+//   - the update from the stored moments (a uniform branch: decode the new
+//     codes again);
+//   - the bf16 copy of the new params (a uniform branch: one 8-byte store
+//     per 4 elements).
+// The ragged end of a chunk and unaligned tensors go through the per-thread
+// element paths of fp8adam_ext.cuh with the same rounding mode.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "fp8_codec.cuh"
+#include "fp8adam_ext.cuh"
+#include "fp8adam_step.cuh"
+#include "fp8adam_step_tma.cuh"
+
+namespace fp8adam {
+
+__device__ __forceinline__ uint32_t bf16_pair(float lo, float hi) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+}
+
+// 4 elements of stage `st` at offset j (global element i, a multiple of 4).
+template <int MF, int VF, bool STATS, bool SR>
+__device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& st, int j, const TensorDesc& td,
+                                             const ExtSeg& sg, int64_t i, float& am, float& av, uint32_t& flushed,
+                                             uint32_t& sat) {
+  const StepConsts& c = a.s.c;
+  const float4 pin = *reinterpret_cast<const float4*>(&st.p[j]);
+  const uint2 gq = *reinterpret_cast<const uint2*>(&st.g[j]);
+  const uint32_t mw = *reinterpret_cast<const uint32_t*>(&st.m[j]);
+  const uint32_t vw = *reinterpret_cast<const uint32_t*>(&st.v[j]);
+  const float2 ma = dec2_hw<MF>(mw & 0xFFFFu), mb = dec2_hw<MF>(mw >> 16);
+  const float2 va = dec2_hw<VF>(vw & 0xFFFFu), vb = dec2_hw<VF>(vw >> 16);
+  const float mo[4] = {__fmul_rn(ma.x, sg.inv_s_m), __fmul_rn(ma.y, sg.inv_s_m), __fmul_rn(mb.x, sg.inv_s_m),
+                       __fmul_rn(mb.y, sg.inv_s_m)};
+  const float vo[4] = {__fmul_rn(va.x, sg.inv_s_v), __fmul_rn(va.y, sg.inv_s_v), __fmul_rn(vb.x, sg.inv_s_v),
+                       __fmul_rn(vb.y, sg.inv_s_v)};
+  const float g[4] = {__fmul_rn(bf16_lo(gq.x), sg.gm), __fmul_rn(bf16_hi(gq.x), sg.gm),
+                      __fmul_rn(bf16_lo(gq.y), sg.gm), __fmul_rn(bf16_hi(gq.y), sg.gm)};
+  const float p4[4] = {pin.x, pin.y, pin.z, pin.w};
+  float mn[4], vn[4], ym[4], yv[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    moments(c, g[e], mo[e], vo[e], mn[e], vn[e]);
+    am = fmax_nan(am, fabsf(mn[e]));
+    av = fmax_nan(av, fabsf(vn[e]));
+    ym[e] = __fmul_rn(mn[e], sg.s_m_new);
+    yv[e] = __fmul_rn(vn[e], sg.s_v_new);
+  }
+  uint32_t mq, vq;
+  if constexpr (SR) {
+    // words of elements (i, i+1) and (i+2, i+3): .x/.y = m/v of the even
+    // element, .z/.w = m/v of the odd one
+    const uint4 r0 = sr_words(a, sg.ti, i >> 1);
+    const uint4 r1 = sr_words(a, sg.ti, (i >> 1) + 1);
+    mq = enc1_sr<MF>(ym[0], r0.x) | (enc1_sr<MF>(ym[1], r0.z) << 8) | (enc1_sr<MF>(ym[2], r1.x) << 16) |
+         (enc1_sr<MF>(ym[3], r1.z) << 24);
+    vq = enc1_sr<VF>(yv[0], r0.y) | (enc1_sr<VF>(yv[1], r0.w) << 8) | (enc1_sr<VF>(yv[2], r1.y) << 16) |
+         (enc1_sr<VF>(yv[3], r1.w) << 24);
+  } else {
+    mq = enc2_hw<MF>(ym[0], ym[1]) | (enc2_hw<MF>(ym[2], ym[3]) << 16);
+    vq = enc2_hw<VF>(yv[0], yv[1]) | (enc2_hw<VF>(yv[2], yv[3]) << 16);
+  }
+  float mu[4] = {mn[0], mn[1], mn[2], mn[3]};
+  float vu[4] = {vn[0], vn[1], vn[2], vn[3]};
+  if (a.flags & kExtFromStored) {  // the update reads the stored values
+    const float2 qa = dec2_hw<MF>(mq & 0xFFFFu), qb = dec2_hw<MF>(mq >> 16);
+    const float2 ra = dec2_hw<VF>(vq & 0xFFFFu), rb = dec2_hw<VF>(vq >> 16);
+    mu[0] = __fmul_rn(qa.x, sg.inv_s_m_new);
+    mu[1] = __fmul_rn(qa.y, sg.inv_s_m_new);
+    mu[2] = __fmul_rn(qb.x, sg.inv_s_m_new);
+    mu[3] = __fmul_rn(qb.y, sg.inv_s_m_new);
+    vu[0] = __fmul_rn(ra.x, sg.inv_s_v_new);
+    vu[1] = __fmul_rn(ra.y, sg.inv_s_v_new);
+    vu[2] = __fmul_rn(rb.x, sg.inv_s_v_new);
+    vu[3] = __fmul_rn(rb.y, sg.inv_s_v_new);
+  }
+  float pout[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) pout[e] = update(c, p4[e], mu[e], vu[e]);
+  if constexpr (STATS) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      sat += fabsf(ym[e]) > FmtTraits<MF>::kMax ? 1u : 0u;
+      sat += fabsf(yv[e]) > FmtTraits<VF>::kMax ? 1u : 0u;
+      flushed += (vn[e] > 0.0f && ((vq >> (8 * e)) & 0x7Fu) == 0u) ? 1u : 0u;
+    }
+  }
+  st_stream_f4(td.p + i, make_float4(pout[0], pout[1], pout[2], pout[3]));
+  __stcs(reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(td.m) + i), mq);
+  __stcs(reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(td.v) + i), vq);
+  if (sg.pb)
+    __stcs(reinterpret_cast<uint2*>(sg.pb + i), make_uint2(bf16_pair(pout[0], pout[1]), bf16_pair(pout[2], pout[3])));
+}
+
+template <int MF, int VF, bool STATS, bool SR>
+__global__ void __launch_bounds__(kThreads, 4)
+fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
+  static_assert(MF != kFP32 && VF != kFP32, "the staged path carries 1-byte codes");
+  extern __shared__ __align__(128) unsigned char tma_smem[];
+  TmaStage* stage = reinterpret_cast<TmaStage*>(tma_smem);
+  __shared__ __align__(8) uint64_t full[kStages];
+  __shared__ uint32_t red[4][kThreads / 32];
+  __shared__ int abort_flag;
+
+  if (*(volatile const uint32_t*)err) return;  // an earlier CTA timed out: stop at once
+  if (a.skip && *a.skip) return;              // a non-finite gradient: the step is skipped
+  const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
+  const Chunk ch = a.s.chunks[blockIdx.x];
+  const int ti = ch.tensor;
+  const TensorDesc td = a.s.tensors[ti];
+  const ExtSeg sg = ext_setup<MF, VF>(a, ti, gm);
+  const int64_t e0 = ch.start, e1 = ch.start + ch.len;
+  float am = 0.0f, av = 0.0f;
+  uint32_t flushed = 0, sat = 0;
+
+  const int nsub = ext_vec_ok(td, sg) ? (int)((e1 - e0) / kSub) : 0;
+  if (!tma_stream(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
+        ext_consume4<MF, VF, STATS, SR>(a, st, j, td, sg, i, am, av, flushed, sat);
+      }))
+    return;
+  // the ragged end (under one sub-tile) or an unaligned tensor, element by element
+  for (int64_t i = e0 + (int64_t)nsub * kSub + threadIdx.x; i < e1; i += kThreads)
+    ext_element<MF, VF, STATS, SR ? kRoundStochastic : kRoundNearest>(a, td, sg, i, am, av, flushed, sat);
+  ext_flush<STATS>(a, ti, td.nunits, sg, am, av, flushed, sat, red);
+}
+
+}  // namespace fp8adam

@@ -120,33 +120,16 @@ __device__ __forceinline__ void consume4(const TmaStage& st, int j, const Tensor
   __stcs(reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(td.v) + i), vq);
 }
 
-template <int MF, int VF, bool STATS>
-__global__ void __launch_bounds__(kThreads, 4)
-fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
-  static_assert(MF != kFP32 && VF != kFP32, "the staged path carries 1-byte codes");
-  extern __shared__ __align__(128) unsigned char tma_smem[];
-  TmaStage* stage = reinterpret_cast<TmaStage*>(tma_smem);
-  __shared__ __align__(8) uint64_t full[kStages];
-  __shared__ uint32_t red[4][kThreads / 32];
-  __shared__ int abort_flag;
-
-  if (*(volatile const uint32_t*)err) return;  // an earlier CTA timed out: stop at once
-  const Chunk ch = a.chunks[blockIdx.x];
-  const int ti = ch.tensor;
-  const TensorDesc td = a.tensors[ti];
-  const StepConsts c = a.c;
-  const int64_t e0 = ch.start, e1 = ch.start + ch.len;
-  const float s_m = a.scale_m[ti];
-  const float s_v = a.scale_v[ti];
-  const float s_m_new = pow2scale<MF>(__uint_as_float(a.amax_in_m[ti]), s_m);
-  const float s_v_new = pow2scale<VF>(__uint_as_float(a.amax_in_v[ti]), s_v);
-  const float inv_s_m = __fdiv_rn(1.0f, s_m);
-  const float inv_s_v = __fdiv_rn(1.0f, s_v);
-  float am = 0.0f, av = 0.0f;
-  uint32_t flushed = 0, sat = 0;
-
-  // whole sub-tiles go through the staged pipeline (aligned tensors only)
-  const int nsub = td.aligned ? (int)((e1 - e0) / kSub) : 0;
+// The staged pipeline over the first nsub whole sub-tiles of the chunk that
+// starts at element e0 of td: thread 0 issues the bulk copies of p, g, m, v
+// into the kStages-deep ring, and every thread calls body(st, j, i) for its
+// 2 groups of 4 elements of each sub-tile (stage st, stage offset j, global
+// element i).  `full` and `abort_flag` live in the kernel's shared memory.
+// Returns false if a wait gave up: then bit 0 of *err is set and the copies
+// still in flight have been waited for (bounded), so the CTA can return.
+template <typename Body>
+__device__ __forceinline__ bool tma_stream(const TensorDesc& td, int64_t e0, int nsub, TmaStage* stage,
+                                           uint64_t* full, int& abort_flag, uint32_t* err, Body&& body) {
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
@@ -176,13 +159,12 @@ fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
         for (int q = k; q < last; ++q) (void)mbar_wait(&full[q % kStages], (uint32_t)((q / kStages) & 1));
       }
       __syncthreads();
-      return;  // the chunk stays unfinished; the host sees the flag
+      return false;  // the chunk stays unfinished; the host sees the flag
     }
 #pragma unroll
     for (int h = 0; h < kSub / (4 * kThreads); ++h) {  // 2 groups of 4 elements per thread
       const int j = h * (4 * kThreads) + 4 * (int)threadIdx.x;
-      consume4<MF, VF, STATS>(stage[s], j, td, e0 + (int64_t)k * kSub + j, c, inv_s_m, inv_s_v, s_m_new, s_v_new,
-                              am, av, flushed, sat);
+      body(stage[s], j, e0 + (int64_t)k * kSub + j);
     }
     __syncthreads();  // every thread is done reading stage s
     if (threadIdx.x == 0 && k + kStages < nsub) {
@@ -190,6 +172,40 @@ fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
       issue(k + kStages);
     }
   }
+  return true;
+}
+
+template <int MF, int VF, bool STATS>
+__global__ void __launch_bounds__(kThreads, 4)
+fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
+  static_assert(MF != kFP32 && VF != kFP32, "the staged path carries 1-byte codes");
+  extern __shared__ __align__(128) unsigned char tma_smem[];
+  TmaStage* stage = reinterpret_cast<TmaStage*>(tma_smem);
+  __shared__ __align__(8) uint64_t full[kStages];
+  __shared__ uint32_t red[4][kThreads / 32];
+  __shared__ int abort_flag;
+
+  if (*(volatile const uint32_t*)err) return;  // an earlier CTA timed out: stop at once
+  const Chunk ch = a.chunks[blockIdx.x];
+  const int ti = ch.tensor;
+  const TensorDesc td = a.tensors[ti];
+  const StepConsts c = a.c;
+  const int64_t e0 = ch.start, e1 = ch.start + ch.len;
+  const float s_m = a.scale_m[ti];
+  const float s_v = a.scale_v[ti];
+  const float s_m_new = pow2scale<MF>(__uint_as_float(a.amax_in_m[ti]), s_m);
+  const float s_v_new = pow2scale<VF>(__uint_as_float(a.amax_in_v[ti]), s_v);
+  const float inv_s_m = __fdiv_rn(1.0f, s_m);
+  const float inv_s_v = __fdiv_rn(1.0f, s_v);
+  float am = 0.0f, av = 0.0f;
+  uint32_t flushed = 0, sat = 0;
+
+  // whole sub-tiles go through the staged pipeline (aligned tensors only)
+  const int nsub = td.aligned ? (int)((e1 - e0) / kSub) : 0;
+  if (!tma_stream(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
+        consume4<MF, VF, STATS>(st, j, td, i, c, inv_s_m, inv_s_v, s_m_new, s_v_new, am, av, flushed, sat);
+      }))
+    return;
 
   // the rest of the chunk (a tensor's ragged end, or an unaligned tensor)
   const int64_t r0 = e0 + (int64_t)nsub * kSub;

@@ -230,6 +230,17 @@ int fp8adam_encode(int32_t fmt, const float* x, uint8_t* out, int64_t n,
 int fp8adam_encode_bits_range(int32_t fmt, uint32_t first, int64_t n,
                               uint8_t* out, int32_t impl, void* cuda_stream);
 
+/* Stochastic rounding with caller-given random words: out[j] = the code of
+ * x[j] rounded to the grid value below |x[j]| (lo) or above it (hi), up iff
+ * r[j]*(hi-lo) < (|x[j]|-lo)*2^32; saturating to the largest finite code;
+ * NaN -> 0x7F.  The encoder of FP8ADAM_FLAG_STOCHASTIC_ROUNDING.  x, r, out
+ * device pointers of n elements; returns INVALID_ARG for n < 0 or a NULL
+ * pointer with n > 0, UNSUPPORTED_FMT for fmt other than E4M3/E5M2.
+ * Source: "随机舍入" in section "应对FP8训练稳定性挑战的策略" of
+ * "FP8训练的稳定性挑战…". */
+int fp8adam_encode_sr(int32_t fmt, const float* x, const uint32_t* r,
+                      uint8_t* out, int64_t n, void* cuda_stream);
+
 /* out[j] = dec(fmt, codes[j]) as fp32. */
 int fp8adam_decode(int32_t fmt, const uint8_t* codes, float* out, int64_t n,
                    int32_t impl, void* cuda_stream);

@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.ref_sr_bits.argtypes = [ctypes.c_uint64, ctypes.c_int32, c_i64, c_i64, c_int]
         L.ref_encode_sr.restype = c_u32
         L.ref_encode_sr.argtypes = [c_int, c_f, c_u32]
+        L.ref_encode_sr_array.restype = None
+        L.ref_encode_sr_array.argtypes = [c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, c_i64]
         L.ref_f32_to_bf16.restype = ctypes.c_uint16
         L.ref_f32_to_bf16.argtypes = [c_f]
         L.ref_f32_to_bf16_array.restype = None
@@ -149,6 +151,16 @@ def sr_bits(seed: int, tensor: int, t: int, j: int, which: int) -> int:
 
 def encode_sr(fmt: int, x: float, r: int) -> int:
     return int(lib().ref_encode_sr(fmt, x, r))
+
+
+def encode_sr_array(fmt: int, x, r) -> np.ndarray:
+    """Codes of x[j] stochastically rounded with the random words r[j]."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    r = np.ascontiguousarray(r, dtype=np.uint32)
+    assert x.shape == r.shape
+    out = np.empty(x.size, np.uint8)
+    lib().ref_encode_sr_array(fmt, _ptr(x), _ptr(r), _ptr(out), x.size)
+    return out
 
 
 def f32_to_bf16(x) -> np.ndarray:

@@ -421,6 +421,12 @@ uint32_t ref_encode_sr(int fmt, float x, uint32_t r) {
   return sign | (up ? hi : lo);
 }
 
+void ref_encode_sr_array(int fmt, const float* x, const uint32_t* r, uint8_t* out, int64_t n) {
+  fpenv_guard g = env_enter();
+  for (int64_t j = 0; j < n; ++j) out[j] = (uint8_t)ref_encode_sr(fmt, x[j], r[j]);
+  env_leave(g);
+}
+
 /* bf16 nearest-even rounding of an fp32 value written from the definition:
  * 8 significant bits, rint() (round half to even) on the scaled significand. */
 uint16_t ref_f32_to_bf16(float x) {

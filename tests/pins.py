@@ -177,3 +177,62 @@ class TorchFakeQuantAdamW:
     @property
     def p(self) -> np.ndarray:
         return self.param.detach().numpy()
+
+
+# ------------------------------------------------------------------ stochastic rounding
+def finite_grid(fmt: int) -> np.ndarray:
+    """The format's non-negative finite values in increasing order, from the
+    torch float8 casts (codes 0x00..0x7F, NaN and inf dropped)."""
+    vals = torch_decode(fmt, torch.arange(128, dtype=torch.int32).to(torch.uint8)).numpy().astype(np.float64)
+    return np.unique(vals[np.isfinite(vals)])
+
+
+def sr_threshold(fmt: int, x: np.ndarray):
+    """For finite |x| below the format's max: (lo, hi, T) with lo <= |x| < hi
+    neighbours on the grid and T = ceil((|x| - lo) / (hi - lo) * 2^32), the
+    number of random words r that round |x| up (r < T).  float64 is exact
+    here: |x| - lo has at most 24 significant bits and hi - lo is a power of
+    two."""
+    grid = finite_grid(fmt)
+    a = np.abs(np.asarray(x, np.float64))
+    k = np.searchsorted(grid, a, side="right") - 1
+    lo, hi = grid[k], grid[k + 1]
+    t = np.ceil((a - lo) / (hi - lo) * 4294967296.0)
+    return lo, hi, t
+
+
+def sr_cases(fmt: int, seed: int):
+    """Adversarial inputs for a stochastic-rounding encoder: every fp32
+    binade from the subnormals to beyond the format's max (edge and random
+    mantissas, both signs), the grid values and their midpoints, and the
+    specials; each finite in-range input with the draws r = T-1 (rounds up),
+    r = T (rounds down) and a random r.  Returns (x, r, want_up) with want_up
+    1/0 where the draw decides it and -1 elsewhere."""
+    rng = np.random.default_rng(seed)
+    bits = []
+    for e in range(0, 146):
+        mant = np.concatenate([[0, 1, 2, 0x3FFFFF, 0x400000, 0x400001, 0x7FFFFE, 0x7FFFFF],
+                               rng.integers(0, 1 << 23, 24)])
+        bits.append((e << 23) | mant)
+    bits = np.concatenate(bits).astype(np.uint32)
+    grid = finite_grid(fmt)
+    extra = np.concatenate([grid, (grid[1:] + grid[:-1]) / 2, [FMAX[fmt], np.nextafter(np.float32(FMAX[fmt]), 0)]])
+    x = np.concatenate([bits.view(np.float32), extra.astype(np.float32)])
+    x = np.concatenate([x, -x])
+    fmax = FMAX[fmt]
+    live = np.isfinite(x) & (np.abs(x) < fmax)
+    xs, rs, up = [], [], []
+    _, _, t = sr_threshold(fmt, np.where(live, x, 0.0))
+    for sel_r, u in ((t - 1, 1), (t, 0)):
+        ok = live & (sel_r >= 0) & (sel_r <= 0xFFFFFFFF)
+        xs.append(x[ok])
+        rs.append(sel_r[ok].astype(np.uint64).astype(np.uint32))
+        up.append(np.full(int(ok.sum()), u, np.int8))
+    xs.append(x)
+    rs.append(rng.integers(0, 1 << 32, x.size, dtype=np.uint64).astype(np.uint32))
+    up.append(np.full(x.size, -1, np.int8))
+    spec = np.array([np.nan, -np.nan, np.inf, -np.inf, 0.0, -0.0, 1e30, -1e30], np.float32)
+    xs.append(spec)
+    rs.append(rng.integers(0, 1 << 32, spec.size, dtype=np.uint64).astype(np.uint32))
+    up.append(np.full(spec.size, -1, np.int8))
+    return np.concatenate(xs).astype(np.float32), np.concatenate(rs), np.concatenate(up)

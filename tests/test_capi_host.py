@@ -73,6 +73,11 @@ def test_step_and_codec_reject_bad_arguments_on_host(L):
     assert L.fp8adam_decode(5, 8, 8, 4, 0, None) == capi.ERR_UNSUPPORTED_FMT
     assert L.fp8adam_encode_bits_range(0, 0xFFFFFFFF, 2, 16, 0, None) == capi.ERR_INVALID_ARG
     assert L.fp8adam_encode_bits_range(0, 0, 4, 2, 0, None) == capi.ERR_INVALID_ARG  # misaligned out
+    assert L.fp8adam_encode_sr(2, 8, 8, 8, 4, None) == capi.ERR_UNSUPPORTED_FMT
+    assert L.fp8adam_encode_sr(0, 8, 8, 8, -1, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_encode_sr(0, None, 8, 8, 4, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_encode_sr(1, 8, None, 8, 4, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_encode_sr(0, 8, 8, 8, 0, None) == capi.OK  # nothing to do
     assert isinstance(capi.fp8adam_launch_count(), int)
 
 

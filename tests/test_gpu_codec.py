@@ -74,3 +74,22 @@ def test_encode_array_ragged(fmt, impl):
     out = torch.empty(n, dtype=torch.uint8, device="cuda")
     capi.fp8adam_encode(fmt, xd.data_ptr(), out.data_ptr(), n, impl, _stream())
     assert (out.cpu().numpy() == oracle.encode(fmt, x)).all()
+
+
+@pytest.mark.parametrize("fmt", [0, 1], ids=["e4m3", "e5m2"])
+def test_stochastic_rounding_encoder(fmt):
+    """The device SR encoder (the one the step uses with stochastic rounding)
+    against the oracle on adversarial inputs: every fp32 binade, grid values
+    and midpoints, specials, and for each in-range input the draws on both
+    sides of its exact threshold."""
+    x, r, _ = pins.sr_cases(fmt, 29)
+    exp = oracle.encode_sr_array(fmt, x, r)
+    dx = torch.from_numpy(x).cuda()
+    dr = torch.from_numpy(r.view(np.int32)).cuda()
+    out = torch.empty(x.size, dtype=torch.uint8, device="cuda")
+    capi.fp8adam_encode_sr(fmt, dx.data_ptr(), dr.data_ptr(), out.data_ptr(), x.size, _stream())
+    got = out.cpu().numpy()
+    nan = np.isnan(x)
+    assert _nan_code(got[nan], fmt).all()
+    d = np.flatnonzero(got[~nan] != exp[~nan])
+    assert d.size == 0, (x[~nan][d[:8]], r[~nan][d[:8]], got[~nan][d[:8]], exp[~nan][d[:8]])

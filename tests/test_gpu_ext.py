@@ -83,8 +83,9 @@ class ExtRun:
                 assert (h.view(np.uint32) == r.hist_m.view(np.uint32)).all(), (i, "hist_m")
 
 
-def test_margin_and_amax_history():
-    r = ExtRun(41, margin_m=1, margin_v=2, amax_history_len=4)
+@pytest.mark.parametrize("tma", [True, False], ids=["staged", "vector"])
+def test_margin_and_amax_history(tma):
+    r = ExtRun(41, margin_m=1, margin_v=2, amax_history_len=4, tma=tma)
     for _ in range(9):
         r.step()
         r.compare()
@@ -108,23 +109,26 @@ def test_update_from_stored_moments(vf):
         r.compare()
 
 
+@pytest.mark.parametrize("tma", [True, False], ids=["staged", "vector"])
 @pytest.mark.parametrize("fmts", [(oracle.E4M3, oracle.E5M2), (oracle.E5M2, oracle.E4M3)], ids=["m4v5", "m5v4"])
-def test_stochastic_rounding(fmts):
-    r = ExtRun(43, mf=fmts[0], vf=fmts[1], stochastic_rounding=True, seed=0x0123456789ABCDEF)
+def test_stochastic_rounding(fmts, tma):
+    r = ExtRun(43, mf=fmts[0], vf=fmts[1], stochastic_rounding=True, seed=0x0123456789ABCDEF, tma=tma)
     for _ in range(5):
         r.step()
         r.compare()
 
 
-def test_bf16_param_copy():
-    r = ExtRun(44, bf16=True)
+@pytest.mark.parametrize("tma", [True, False], ids=["staged", "vector"])
+def test_bf16_param_copy(tma):
+    r = ExtRun(44, bf16=True, tma=tma)
     for _ in range(3):
         r.step()
         r.compare()
 
 
-def test_loss_scale_clip_and_skip():
-    r = ExtRun(45)
+@pytest.mark.parametrize("tma", [True, False], ids=["staged", "vector"])
+def test_loss_scale_clip_and_skip(tma):
+    r = ExtRun(45, tma=tma)
     for ls, mx in ((1024.0, 1.0), (1.0, 0.05), (65536.0, 0.0), (8.0, 1e-4)):
         norm, skip = r.step(loss_scale=ls, max_norm=mx, skip_nonfinite=True)
         r.compare()
@@ -159,3 +163,38 @@ def test_options_with_fp32_moments_and_current_scaling():
     for _ in range(4):
         r.step(loss_scale=4.0, max_norm=0.5)
         r.compare()
+
+
+def test_options_on_misaligned_views():
+    """Buffers (and the bf16 outputs) that start one element into their
+    allocation take the element-by-element path of the staged variant
+    kernel; stochastic rounding, a margin, the history and the bf16 copy must
+    still match the oracle bit for bit."""
+    dev = torch.device("cuda:0")
+    ns = [33, 4097, 70000]
+    p = [torch.zeros(n + 1, device=dev)[1:] for n in ns]
+    g = [torch.zeros(n + 1, device=dev, dtype=torch.bfloat16)[1:] for n in ns]
+    m = [torch.zeros(n + 1, device=dev, dtype=torch.uint8)[1:] for n in ns]
+    v = [torch.zeros(n + 1, device=dev, dtype=torch.uint8)[1:] for n in ns]
+    pb = [torch.zeros(n + 1, device=dev, dtype=torch.bfloat16)[1:] for n in ns]
+    specs = workloads.custom_layout(ns)
+    workloads.init_params_into(specs, p, 49)
+    kw = dict(stochastic_rounding=True, seed=99, margin_m=1, amax_history_len=3)
+    opt = FP8AdamW(p, g, m=m, v=v, param_bf16=pb, **kw)
+    ref = [oracle.TensorState(x.cpu().numpy(), oracle.E4M3, oracle.E5M2) for x in p]
+    sig = workloads.tensor_sigmas(specs, 49)
+    flags = oracle.FLAG_STOCHASTIC
+    for t in range(1, 5):
+        workloads.grads_into(specs, g, 49, t, sig)
+        opt.step(loss_scale=2.0)
+        grads = [bf16_host_bits(x) for x in g]
+        sumsq, _ = oracle.grad_sumsq(grads)
+        gm = oracle.grad_multiplier(sumsq, 2.0, 0.0)
+        for i, rs in enumerate(ref):
+            rs.step_ex(grads[i], HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], t, flags,
+                       margin_m=1, hist_len=3, seed=99, tensor_index=i, grad_mult=gm, want_bf16=True)
+    torch.cuda.synchronize()
+    for i, rs in enumerate(ref):
+        assert (m[i].cpu().numpy() == rs.m).all() and (v[i].cpu().numpy() == rs.v).all(), i
+        assert (p[i].cpu().numpy().view(np.uint32) == rs.p.view(np.uint32)).all(), i
+        assert (pb[i].cpu().view(torch.int16).numpy().view(np.uint16) == rs.p_bf16).all(), i

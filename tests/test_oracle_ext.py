@@ -305,3 +305,28 @@ def test_stochastic_rounding_step_codes(orc):
             assert q[j] == orc.encode_sr(fmt, float(xs[j]), r)
     # the update itself does not depend on the rounding mode (R2)
     assert (sr.p.view(np.uint32) == fp.p.view(np.uint32)).all()
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2], ids=["e4m3", "e5m2"])
+def test_sr_threshold_is_exact(orc, fmt):
+    """At the draw r = T - 1 the oracle rounds up to hi, at r = T down to lo,
+    T = ceil((|x|-lo)/(hi-lo) * 2^32) computed in float64 from the torch
+    float8 grid; out of range and non-finite inputs saturate or give NaN."""
+    x, r, want_up = pins.sr_cases(fmt, 17)
+    got = orc.encode_sr_array(fmt, x, r)
+    decided = want_up >= 0
+    lo, hi, _ = pins.sr_threshold(fmt, x[decided])
+    val = np.abs(orc.decode(fmt, got[decided] & 0x7F).astype(np.float64))
+    assert (val == np.where(want_up[decided] == 1, hi, lo)).all()
+    assert ((got[decided] >> 7) == np.signbit(x[decided])).all()
+    # every code is one of the two neighbours (or the saturated / NaN code)
+    fin = np.isfinite(x) & (np.abs(x) < pins.FMAX[fmt])
+    lo, hi, _ = pins.sr_threshold(fmt, np.where(fin, x, 0.0))
+    v = np.abs(orc.decode(fmt, got & 0x7F).astype(np.float64))
+    assert ((v == lo) | (v == hi))[fin].all()
+    big = ~np.isnan(x) & (np.abs(x) >= pins.FMAX[fmt])
+    assert (v[big] == pins.FMAX[fmt]).all()
+    assert ((got[np.isnan(x)] & 0x7F) == 0x7F).all()
+    # the array form is the scalar encoder element by element
+    for j in range(0, x.size, 97):
+        assert got[j] == orc.encode_sr(fmt, float(x[j]), int(r[j]))
