@@ -470,8 +470,10 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
   e.hist_slot = ctx->hist_len ? (int32_t)((p.step - 1) % ctx->hist_len) : 0;
   e.hist_m = ctx->hist_m;
   e.hist_v = ctx->hist_v;
-  e.seed_lo = (uint32_t)ctx->seed;
-  e.seed_hi = (uint32_t)(ctx->seed >> 32);
+  for (int r = 0; r < 10; ++r) {  // Philox4x32-10 key schedule (Weyl increments)
+    e.sr_key[r][0] = (uint32_t)ctx->seed + (uint32_t)r * 0x9E3779B9u;
+    e.sr_key[r][1] = (uint32_t)(ctx->seed >> 32) + (uint32_t)r * 0xBB67AE85u;
+  }
   e.t_lo = (uint32_t)p.step;
   e.grad_mult = nullptr;
   e.skip = nullptr;

@@ -38,34 +38,54 @@ struct ExtArgs {
   int32_t hist_slot;        // this step's slot, (t-1) % hist_len
   float* hist_m;            // [hist_len][T] or null
   float* hist_v;
-  uint32_t seed_lo, seed_hi, t_lo;
+  uint32_t sr_key[10][2];    // Philox round keys: round r uses seed + r * (0x9E3779B9, 0xBB67AE85)
+  uint32_t t_lo;             // the step (counter word 3)
   const float* grad_mult;   // device scalar, or null (1.0)
   const uint32_t* skip;     // device flag, or null
   uint16_t* const* p_bf16;  // device array [T] of bf16 outputs (entries may be null), or null
 };
 
 // ------------------------------------------------------------ Philox4x32-10
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
-#pragma unroll
-  for (int r = 0; r < 10; ++r) {
-    if (r > 0) {
-      k0 += 0x9E3779B9u;
-      k1 += 0xBB67AE85u;
-    }
-    const uint32_t lo0 = 0xD2511F53u * c.x;
-    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x);
-    const uint32_t lo1 = 0xCD9E8D57u * c.z;
-    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z);
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
-  }
-  return c;
+constexpr uint32_t kPhiloxM0 = 0xD2511F53u, kPhiloxM1 = 0xCD9E8D57u;
+
+// One round: each product as one 32 x 32 -> 64-bit multiply (low and high
+// words together).
+__device__ __forceinline__ uint4 philox_round(uint4 c, uint32_t k0, uint32_t k1) {
+  const uint64_t p0 = (uint64_t)kPhiloxM0 * c.x;
+  const uint64_t p1 = (uint64_t)kPhiloxM1 * c.z;
+  return make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ k0, (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ k1, (uint32_t)p0);
 }
 
 // random words of elements (2q, 2q+1) of tensor ti at this step:
 // .x/.y -> element 2q (m, v); .z/.w -> element 2q+1 (m, v)
 __device__ __forceinline__ uint4 sr_words(const ExtArgs& a, int ti, int64_t q) {
-  return philox4x32_10(make_uint4((uint32_t)q, (uint32_t)((uint64_t)q >> 32), (uint32_t)ti, a.t_lo), a.seed_lo,
-                       a.seed_hi);
+  uint4 c = make_uint4((uint32_t)q, (uint32_t)((uint64_t)q >> 32), (uint32_t)ti, a.t_lo);
+#pragma unroll
+  for (int r = 0; r < 10; ++r) c = philox_round(c, a.sr_key[r][0], a.sr_key[r][1]);
+  return c;
+}
+
+// The same words within one chunk.  A chunk never crosses a multiple of
+// 2^33 elements (its start is a multiple of its power-of-two length), so the
+// counter's words 1..3 are the same for all its pairs, and so is half of the
+// first round's output: computed once per chunk.
+struct SrChunk {
+  uint32_t x1, y1, w1;
+};
+__device__ __forceinline__ SrChunk sr_chunk(const ExtArgs& a, int ti, int64_t q0) {
+  const uint64_t p1 = (uint64_t)kPhiloxM1 * (uint32_t)ti;
+  SrChunk u;
+  u.x1 = (uint32_t)(p1 >> 32) ^ (uint32_t)((uint64_t)q0 >> 32) ^ a.sr_key[0][0];
+  u.y1 = (uint32_t)p1;
+  u.w1 = a.t_lo ^ a.sr_key[0][1];
+  return u;
+}
+__device__ __forceinline__ uint4 sr_words_chunk(const ExtArgs& a, const SrChunk& u, uint32_t q_lo) {
+  const uint64_t p0 = (uint64_t)kPhiloxM0 * q_lo;
+  uint4 c = make_uint4(u.x1, u.y1, (uint32_t)(p0 >> 32) ^ u.w1, (uint32_t)p0);
+#pragma unroll
+  for (int r = 1; r < 10; ++r) c = philox_round(c, a.sr_key[r][0], a.sr_key[r][1]);
+  return c;
 }
 
 // ------------------------------------------------------------ SR encoder

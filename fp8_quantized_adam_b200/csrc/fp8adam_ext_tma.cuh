@@ -36,8 +36,8 @@ __device__ __forceinline__ uint32_t bf16_pair(float lo, float hi) {
 // 4 elements of stage `st` at offset j (global element i, a multiple of 4).
 template <int MF, int VF, bool STATS, bool SR>
 __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& st, int j, const TensorDesc& td,
-                                             const ExtSeg& sg, int64_t i, float& am, float& av, uint32_t& flushed,
-                                             uint32_t& sat) {
+                                             const ExtSeg& sg, const SrChunk& su, int64_t i, float& am, float& av,
+                                             uint32_t& flushed, uint32_t& sat) {
   const StepConsts& c = a.s.c;
   const float4 pin = *reinterpret_cast<const float4*>(&st.p[j]);
   const uint2 gq = *reinterpret_cast<const uint2*>(&st.g[j]);
@@ -65,8 +65,8 @@ __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& s
   if constexpr (SR) {
     // words of elements (i, i+1) and (i+2, i+3): .x/.y = m/v of the even
     // element, .z/.w = m/v of the odd one
-    const uint4 r0 = sr_words(a, sg.ti, i >> 1);
-    const uint4 r1 = sr_words(a, sg.ti, (i >> 1) + 1);
+    const uint4 r0 = sr_words_chunk(a, su, (uint32_t)(i >> 1));
+    const uint4 r1 = sr_words_chunk(a, su, (uint32_t)(i >> 1) + 1u);
     mq = enc1_sr<MF>(ym[0], r0.x) | (enc1_sr<MF>(ym[1], r0.z) << 8) | (enc1_sr<MF>(ym[2], r1.x) << 16) |
          (enc1_sr<MF>(ym[3], r1.z) << 24);
     vq = enc1_sr<VF>(yv[0], r0.y) | (enc1_sr<VF>(yv[1], r0.w) << 8) | (enc1_sr<VF>(yv[2], r1.y) << 16) |
@@ -128,9 +128,11 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   float am = 0.0f, av = 0.0f;
   uint32_t flushed = 0, sat = 0;
 
+  SrChunk su{0u, 0u, 0u};
+  if constexpr (SR) su = sr_chunk(a, ti, e0 >> 1);
   const int nsub = ext_vec_ok(td, sg) ? (int)((e1 - e0) / kSub) : 0;
   if (!tma_stream(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
-        ext_consume4<MF, VF, STATS, SR>(a, st, j, td, sg, i, am, av, flushed, sat);
+        ext_consume4<MF, VF, STATS, SR>(a, st, j, td, sg, su, i, am, av, flushed, sat);
       }))
     return;
   // the ragged end (under one sub-tile) or an unaligned tensor, element by element
