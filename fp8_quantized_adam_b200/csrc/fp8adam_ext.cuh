@@ -91,31 +91,36 @@ __device__ __forceinline__ uint4 sr_words_chunk(const ExtArgs& a, const SrChunk&
 // ------------------------------------------------------------ SR encoder
 // Round up to the next grid value iff r < (|x| - lo) / (hi - lo) * 2^32 (that
 // is r * (hi - lo) < (|x| - lo) * 2^32); saturate; NaN -> 0x7F.
+//
+// On the normal grid (2^emin <= |x| < max), the common case, one range test
+// selects the integer path: the spacing is 2^sh fp32 ulps of |x|, the code
+// is |x|'s bits shifted right by sh (rebiased), and the condition is exactly
+// "the top 32 - sh bits of r are below the sh dropped bits".  Below 2^emin
+// the spacing is fixed: y = |x| / spacing is exact, and the threshold is
+// ceil(frac(y) * 2^32).  (Adding 2^emin with round-toward-zero instead, to
+// reuse the integer test, was measured slower.)
 template <int FMT>
 __device__ __forceinline__ uint32_t enc1_sr(float x, uint32_t r) {
   using T = FmtTraits<FMT>;
+  constexpr int sh = 23 - T::kMant;
+  constexpr uint32_t kMinNormal = (uint32_t)(127 + 1 - T::kBias) << 23;  // bits of 2^emin
   const uint32_t u = __float_as_uint(x);
-  const uint32_t sign = (u >> 24) & 0x80u;
   const uint32_t a = u & 0x7FFFFFFFu;
-  if (a > 0x7F800000u) return 0x7Fu;
-  if (a >= T::kMaxBits) return sign | T::kMaxCode;
-  const uint32_t min_normal = (uint32_t)(127 + 1 - T::kBias) << 23;
   uint32_t code;
-  if (a < min_normal) {
-    // y = |x| / (quantum 2^(1-bias-M)), exact; n = floor(y), f = y - n exact
+  if (a - kMinNormal < T::kMaxBits - kMinNormal) {  // normal grid, below the max
+    code = ((a - kMinNormal) >> sh) + (1u << T::kMant) + ((r >> (32 - sh)) < (a & ((1u << sh) - 1u)) ? 1u : 0u);
+  } else if (a >= T::kMaxBits) {                     // saturate, or NaN
+    if (a > 0x7F800000u) return 0x7Fu;
+    code = T::kMaxCode;
+  } else {                                           // below 2^emin
+    // y = |x| / (spacing 2^(1-bias-M)), exact; n = floor(y), f = y - n exact
     const float y = __fmul_rn(__uint_as_float(a), __uint_as_float((uint32_t)(127 + T::kBias - 1 + T::kMant) << 23));
     const float n = floorf(y);
     const float f = __fsub_rn(y, n);
     const uint32_t thr = __float2uint_ru(__fmul_rn(f, 4294967296.0f));  // ceil(f * 2^32); the product is exact
     code = (uint32_t)n + (r < thr ? 1u : 0u);
-  } else {
-    // quantum = 2^sh fp32 ulps: keep the truncated bits, round up iff the
-    // top (32 - sh) bits of r are below the dropped bits
-    constexpr int sh = 23 - T::kMant;
-    const uint32_t dropped = a & ((1u << sh) - 1u);
-    code = (a >> sh) + ((r >> (32 - sh)) < dropped ? 1u : 0u) - ((uint32_t)(127 - T::kBias) << T::kMant);
   }
-  return sign | code;
+  return ((u >> 24) & 0x80u) | code;
 }
 
 // ------------------------------------------------------------ scale with margin

@@ -33,6 +33,11 @@ __device__ __forceinline__ uint32_t bf16_pair(float lo, float hi) {
          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
 }
 
+// four codes (each < 256) into one word, byte k = ck
+__device__ __forceinline__ uint32_t pack4(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3) {
+  return __byte_perm(__byte_perm(c0, c1, 0x7740), __byte_perm(c2, c3, 0x7740), 0x5410);
+}
+
 // 4 elements of stage `st` at offset j (global element i, a multiple of 4).
 template <int MF, int VF, bool STATS, bool SR>
 __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& st, int j, const TensorDesc& td,
@@ -67,10 +72,10 @@ __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& s
     // element, .z/.w = m/v of the odd one
     const uint4 r0 = sr_words_chunk(a, su, (uint32_t)(i >> 1));
     const uint4 r1 = sr_words_chunk(a, su, (uint32_t)(i >> 1) + 1u);
-    mq = enc1_sr<MF>(ym[0], r0.x) | (enc1_sr<MF>(ym[1], r0.z) << 8) | (enc1_sr<MF>(ym[2], r1.x) << 16) |
-         (enc1_sr<MF>(ym[3], r1.z) << 24);
-    vq = enc1_sr<VF>(yv[0], r0.y) | (enc1_sr<VF>(yv[1], r0.w) << 8) | (enc1_sr<VF>(yv[2], r1.y) << 16) |
-         (enc1_sr<VF>(yv[3], r1.w) << 24);
+    mq = pack4(enc1_sr<MF>(ym[0], r0.x), enc1_sr<MF>(ym[1], r0.z), enc1_sr<MF>(ym[2], r1.x),
+               enc1_sr<MF>(ym[3], r1.z));
+    vq = pack4(enc1_sr<VF>(yv[0], r0.y), enc1_sr<VF>(yv[1], r0.w), enc1_sr<VF>(yv[2], r1.y),
+               enc1_sr<VF>(yv[3], r1.w));
   } else {
     mq = enc2_hw<MF>(ym[0], ym[1]) | (enc2_hw<MF>(ym[2], ym[3]) << 16);
     vq = enc2_hw<VF>(yv[0], yv[1]) | (enc2_hw<VF>(yv[2], yv[3]) << 16);
