@@ -41,12 +41,12 @@ FALLBACK_HBM_GBS = 6650.0
 # from the ncu capture summarised in profiles/, valid while the kernel sources
 # hash to KERNEL_SHA (null otherwise).
 TRAFFIC_PER_PARAM = 13.4719  # profiles/fp8adam_step_tma_kernel_llama2_100m.md: 876.40 MB + 599.16 MB / 109.53 M
-KERNEL_SHA = "b9f75aa41e53ac98"
+KERNEL_SHA = "f5fd7065a55be140"
 
 
 def kernel_sha() -> str:
     h = hashlib.sha256()
-    for f in ("fp8adam_step.cuh", "fp8adam_step_tma.cuh", "fp8_codec.cuh", "fp8adam_capi.cu"):
+    for f in ("fp8adam_step.cuh", "fp8adam_step_tma.cuh", "fp8_codec.cuh"):  # the step kernel's device code
         with open(os.path.join(ROOT, "fp8_quantized_adam_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -291,18 +291,21 @@ def our_arm(args):
             e2e_steps = max(1, min(args.steps, args.e2e_steps))
             barrier()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            host_views = [g_host[o:o + sp.numel] for o, sp in zip(model.off, specs)]
             e0.record(stream)
             for _ in range(e2e_steps):
-                model.g.copy_(g_host, non_blocking=True)
-                opt.step(**step_kw)
-                am_host[:len(specs)].copy_(model.amax_m, non_blocking=True)
-                am_host[len(specs):].copy_(model.amax_v, non_blocking=True)
+                # the library copies each tensor's gradients from the pinned
+                # host buffer and steps each group of tensors as it arrives;
+                # the step's amax comes back to the host
+                opt.step_host(host_views, am_host, stream=stream, **step_kw)
             e1.record(stream)
             barrier()
             et = ranks.max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
             e2e = {"value": world * n_params * e2e_steps / et, "unit": UNIT,
-                   "h2d_bytes_per_step": g_host.numel() * g_host.element_size(),
-                   "d2h_bytes_per_step": am_host.numel() * am_host.element_size(), "steps": e2e_steps}
+                   "h2d_bytes_per_step": 2 * n_params,
+                   "d2h_bytes_per_step": am_host.numel() * am_host.element_size(), "steps": e2e_steps,
+                   "api": "FP8AdamW.step_host -> fp8adam_step_host (per-tensor H2D copies on the library's copy "
+                          "stream, overlapping the step of earlier tensor groups)"}
         elif e2e is None:
             e2e = {"value": None, "unit": UNIT, "unavailable": "pinned host buffer refused on another rank"}
         del g_host

@@ -86,6 +86,9 @@ def lib() -> ctypes.CDLL:
         L.fp8adam_encode_bits_range.argtypes = [i32, u32, i64, vp, i32, vp]
         L.fp8adam_decode.restype = ctypes.c_int
         L.fp8adam_decode.argtypes = [i32, vp, vp, i64, i32, vp]
+        L.fp8adam_step_host.restype = ctypes.c_int
+        L.fp8adam_step_host.argtypes = [vp, ctypes.POINTER(fp8adam_step_params), ctypes.POINTER(ctypes.c_void_p),
+                                        vp, vp]
         L.fp8adam_encode_sr.restype = ctypes.c_int
         L.fp8adam_encode_sr.argtypes = [i32, vp, vp, vp, i64, vp]
         L.fp8adam_launch_count.restype = ctypes.c_uint64
@@ -175,6 +178,12 @@ def fp8adam_encode_bits_range(fmt: int, first: int, n: int, out: int, impl: int,
     _check("fp8adam_encode_bits_range", lib().fp8adam_encode_bits_range(fmt, first, n, out, impl, cuda_stream))
 
 
+def fp8adam_step_host(ctx, params: fp8adam_step_params, host_grads, amax_host: int, cuda_stream: int) -> None:
+    """host_grads: a ctypes array of host pointers, one per tensor."""
+    _check("fp8adam_step_host", lib().fp8adam_step_host(ctx, ctypes.byref(params), host_grads, amax_host or None,
+                                                        cuda_stream))
+
+
 def fp8adam_encode_sr(fmt: int, x: int, r: int, out: int, n: int, cuda_stream: int) -> None:
     _check("fp8adam_encode_sr", lib().fp8adam_encode_sr(fmt, x, r, out, n, cuda_stream))
 
@@ -200,4 +209,4 @@ def fp8adam_step_noalloc(tensors, num_tensors: int, scale_m: int, scale_v: int, 
 EXPORTED = ["fp8adam_create", "fp8adam_step", "fp8adam_get_stats", "fp8adam_reset_stats",
             "fp8adam_destroy", "fp8adam_strerror", "fp8adam_encode", "fp8adam_encode_bits_range",
             "fp8adam_decode", "fp8adam_launch_count", "fp8adam_step_noalloc", "fp8adam_create_ex",
-            "fp8adam_step_ex", "fp8adam_get_grad_info", "fp8adam_check", "fp8adam_encode_sr"]
+            "fp8adam_step_ex", "fp8adam_get_grad_info", "fp8adam_check", "fp8adam_encode_sr", "fp8adam_step_host"]

@@ -213,6 +213,16 @@ struct fp8adam_ctx {
   double* d_norm = nullptr;
   uint32_t* d_state = nullptr;  // [5T]: acc_m, acc_v, jit_m, jit_v, done
   unsigned long long* d_stats = nullptr;
+  // fp8adam_step_host: each tensor's device gradient buffer and size, and
+  // the tensor groups (cut at tensor boundaries, about equal in elements)
+  // whose steps overlap the copies of the groups after them
+  std::vector<uint16_t*> grad_dev;    // [T]
+  std::vector<int64_t> numel;         // [T]
+  std::vector<int32_t> grp_tensor;    // [G+1] first tensor of each group
+  std::vector<int32_t> grp_chunk;     // [G+1] first chunk of each group
+  cudaStream_t copy_stream = nullptr; // created on first use
+  cudaEvent_t start_event = nullptr;
+  std::vector<cudaEvent_t> grp_event; // [G] the group's copies are done
 };
 
 static void free_ctx(fp8adam_ctx* c) {
@@ -228,6 +238,10 @@ static void free_ctx(fp8adam_ctx* c) {
   cudaFree(c->d_norm);
   cudaFree(c->d_state);
   cudaFree(c->d_stats);
+  for (cudaEvent_t e : c->grp_event)
+    if (e) cudaEventDestroy(e);
+  if (c->start_event) cudaEventDestroy(c->start_event);
+  if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
   delete c;
 }
 
@@ -316,6 +330,34 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
 
   fp8adam_ctx* c = new (std::nothrow) fp8adam_ctx();
   if (!c) return FP8ADAM_ERR_OOM;
+  try {
+    c->grad_dev.resize((size_t)num_tensors);
+    c->numel.resize((size_t)num_tensors);
+    int64_t total_elems = 0;
+    for (int32_t i = 0; i < num_tensors; ++i) {
+      c->grad_dev[(size_t)i] = const_cast<uint16_t*>(tensors[i].grad);
+      c->numel[(size_t)i] = tensors[i].numel;
+      total_elems += tensors[i].numel;
+    }
+    // groups for fp8adam_step_host: up to kHostGroups, cut after the tensor
+    // that reaches the next equal share of the elements
+    constexpr int kHostGroups = 8;
+    c->grp_tensor.push_back(0);
+    c->grp_chunk.push_back(0);
+    int64_t cum = 0, cum_chunks = 0;
+    for (int32_t i = 0; i < num_tensors; ++i) {
+      cum += tensors[i].numel;
+      cum_chunks += (tensors[i].numel + chunk - 1) / chunk;
+      const int g = (int)c->grp_tensor.size();  // groups closed so far + 1
+      if (i + 1 == num_tensors || (g < kHostGroups && cum * kHostGroups >= total_elems * g)) {
+        c->grp_tensor.push_back(i + 1);
+        c->grp_chunk.push_back((int32_t)cum_chunks);
+      }
+    }
+  } catch (...) {
+    delete c;
+    return FP8ADAM_ERR_OOM;
+  }
   c->device = dev;
   c->chunk_elems = (int32_t)chunk;
   c->T = num_tensors;
@@ -396,12 +438,19 @@ static bool valid_hparams(float lr, float beta1, float beta2, float eps, float w
          beta2 >= 0.0f && beta2 < 1.0f && eps >= 0.0f && std::isfinite(eps);
 }
 
-static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t st) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FP8ADAM_ERR_CUDA;
-  if (dev != ctx->device) return FP8ADAM_ERR_WRONG_DEVICE;
-  if (ctx->total_units == 0) return FP8ADAM_OK;  // every tensor empty
-  const bool prepass = p.loss_scale != 1.0f || p.max_norm > 0.0f || p.skip_nonfinite != 0;
+static bool needs_prepass(const fp8adam_step_params& p) {
+  return p.loss_scale != 1.0f || p.max_norm > 0.0f || p.skip_nonfinite != 0;
+}
+
+// The step over chunks [c0, c1) of the chunk table: every chunk of the
+// tensors in that range (ranges start and end at tensor boundaries).
+// `first`: the range is the step's first, so the JIT accumulators are
+// cleared before it.  The grad-norm pre-pass needs all gradients: with it
+// the range is the whole table.
+static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t st, int32_t c0, int32_t c1,
+                          bool first) {
+  if (c1 <= c0) return FP8ADAM_OK;  // only empty tensors
+  const bool prepass = needs_prepass(p);
   const bool ext = ctx->ext || prepass;
 
   // constants of step t: double, rounded once to fp32
@@ -423,7 +472,7 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
   uint32_t* jit_m = ctx->d_state + 2 * T;
   uint32_t* jit_v = ctx->d_state + 3 * T;
   a.tensors = ctx->d_tensors;
-  a.chunks = ctx->d_chunks;
+  a.chunks = ctx->d_chunks + c0;
   a.num_tensors = ctx->T;
   a.scale_m = ctx->scale_m;
   a.scale_v = ctx->scale_v;
@@ -434,12 +483,12 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
   a.acc_m = acc_m;
   a.acc_v = acc_v;
 
-  const dim3 block(kThreads), grid((unsigned)ctx->total_units);
+  const dim3 block(kThreads), grid((unsigned)(c1 - c0));
   const bool jit = p.step == 1 || (ctx->flags & FP8ADAM_FLAG_JIT_EVERY_STEP);
   const bool stats = (ctx->flags & FP8ADAM_FLAG_STATS) != 0;
   if (!ext) {
     if (jit) {
-      if (cudaMemsetAsync(jit_m, 0, 2 * T * sizeof(uint32_t), st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
+      if (first && cudaMemsetAsync(jit_m, 0, 2 * T * sizeof(uint32_t), st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
       StepArgs pre = a;
       pre.acc_m = jit_m;
       pre.acc_v = jit_v;
@@ -482,7 +531,7 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
     if (cudaMemsetAsync(ctx->d_nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)
       return FP8ADAM_ERR_CUDA;
     fp8adam_gradnorm_partial_kernel<<<grid, block, 0, st>>>(a, ctx->d_partial, ctx->d_nonfinite);
-    fp8adam_gradnorm_finalize_kernel<<<1, block, 0, st>>>(ctx->d_partial, ctx->total_units, ctx->d_nonfinite,
+    fp8adam_gradnorm_finalize_kernel<<<1, block, 0, st>>>(ctx->d_partial, (int)(c1 - c0), ctx->d_nonfinite,
                                                           p.loss_scale, p.max_norm, p.skip_nonfinite,
                                                           ctx->d_grad_mult, ctx->d_skip, ctx->d_norm);
     g_launches.fetch_add(2, std::memory_order_relaxed);
@@ -490,7 +539,7 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
     e.skip = ctx->d_skip;
   }
   if (jit) {
-    if (cudaMemsetAsync(jit_m, 0, 2 * T * sizeof(uint32_t), st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
+    if (first && cudaMemsetAsync(jit_m, 0, 2 * T * sizeof(uint32_t), st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
     ExtArgs pre = e;
     pre.s = a;
     pre.s.acc_m = jit_m;
@@ -513,6 +562,13 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
     pick_ext(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return last_error();
+}
+
+static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t st) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP8ADAM_ERR_CUDA;
+  if (dev != ctx->device) return FP8ADAM_ERR_WRONG_DEVICE;
+  return run_step_range(ctx, p, st, 0, ctx->total_units, true);
 }
 
 extern "C" int fp8adam_step(fp8adam_ctx* ctx, float lr, float beta1, float beta2, float eps,
@@ -540,6 +596,69 @@ extern "C" int fp8adam_step_ex(fp8adam_ctx* ctx, const fp8adam_step_params* para
       std::isinf(p.max_norm))
     return FP8ADAM_ERR_INVALID_ARG;
   return run_step(ctx, p, static_cast<cudaStream_t>(cuda_stream));
+}
+
+extern "C" int fp8adam_step_host(fp8adam_ctx* ctx, const fp8adam_step_params* params,
+                                 const uint16_t* const* host_grads, float* amax_host, void* cuda_stream) {
+  if (!ctx || !params || !host_grads) return FP8ADAM_ERR_INVALID_ARG;
+  const fp8adam_step_params& p = *params;
+  if (!valid_hparams(p.lr, p.beta1, p.beta2, p.eps, p.weight_decay, p.step)) return FP8ADAM_ERR_INVALID_ARG;
+  if (!(p.loss_scale > 0.0f) || !std::isfinite(p.loss_scale) || std::isnan(p.max_norm) ||
+      std::isinf(p.max_norm))
+    return FP8ADAM_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < ctx->T; ++i)
+    if (ctx->numel[(size_t)i] > 0 && !host_grads[i]) return FP8ADAM_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP8ADAM_ERR_CUDA;
+  if (dev != ctx->device) return FP8ADAM_ERR_WRONG_DEVICE;
+  const int G = (int)ctx->grp_tensor.size() - 1;
+  if (!ctx->copy_stream) {  // first use: the copy stream and its events
+    if (cudaStreamCreateWithFlags(&ctx->copy_stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ctx->start_event, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      return FP8ADAM_ERR_CUDA;
+    }
+    ctx->grp_event.assign((size_t)G, nullptr);
+    for (int g = 0; g < G; ++g)
+      if (cudaEventCreateWithFlags(&ctx->grp_event[(size_t)g], cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8ADAM_ERR_CUDA;
+      }
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  // the copies wait for the work already queued on the step's stream (the
+  // previous step may still read the gradient buffers)
+  if (cudaEventRecord(ctx->start_event, st) != cudaSuccess ||
+      cudaStreamWaitEvent(ctx->copy_stream, ctx->start_event, 0) != cudaSuccess)
+    return FP8ADAM_ERR_CUDA;
+  // with the grad-norm pre-pass every gradient is needed before any update:
+  // one group; otherwise group g's step waits only for group g's copies
+  const bool whole = needs_prepass(p);
+  const int ng = whole ? 1 : G;
+  for (int g = 0; g < ng; ++g) {
+    const int32_t t0 = whole ? 0 : ctx->grp_tensor[(size_t)g];
+    const int32_t t1 = whole ? ctx->T : ctx->grp_tensor[(size_t)g + 1];
+    for (int32_t i = t0; i < t1; ++i) {
+      const int64_t n = ctx->numel[(size_t)i];
+      if (n > 0 && cudaMemcpyAsync(ctx->grad_dev[(size_t)i], host_grads[i], (size_t)n * sizeof(uint16_t),
+                                   cudaMemcpyHostToDevice, ctx->copy_stream) != cudaSuccess)
+        return FP8ADAM_ERR_CUDA;
+    }
+    cudaEvent_t ev = ctx->grp_event[(size_t)g];
+    if (cudaEventRecord(ev, ctx->copy_stream) != cudaSuccess || cudaStreamWaitEvent(st, ev, 0) != cudaSuccess)
+      return FP8ADAM_ERR_CUDA;
+    const int32_t c0 = whole ? 0 : ctx->grp_chunk[(size_t)g];
+    const int32_t c1 = whole ? ctx->total_units : ctx->grp_chunk[(size_t)g + 1];
+    const int rc = run_step_range(ctx, p, st, c0, c1, g == 0);
+    if (rc != FP8ADAM_OK) return rc;
+  }
+  if (amax_host && ctx->T > 0) {
+    const size_t bytes = (size_t)ctx->T * sizeof(float);
+    if (cudaMemcpyAsync(amax_host, ctx->amax_m, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(amax_host + ctx->T, ctx->amax_v, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return FP8ADAM_ERR_CUDA;
+  }
+  return last_error();
 }
 
 extern "C" int fp8adam_get_grad_info(fp8adam_ctx* ctx, double* grad_norm, uint32_t* skipped, void* cuda_stream) {

@@ -123,6 +123,41 @@ class FP8AdamW:
                                           loss_scale, max_norm, 1 if skip_nonfinite else 0)
             capi.fp8adam_step_ex(self.ctx, sp, s.cuda_stream)
 
+    def step_host(self, host_grads: Sequence[torch.Tensor], amax_out: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None, lr: Optional[float] = None,
+                  loss_scale: float = 1.0, max_norm: float = 0.0, skip_nonfinite: bool = False) -> None:
+        """One step whose gradients come from host memory: ``host_grads[i]``
+        (a CPU bf16 tensor of tensor i's size, pinned for overlap) is copied
+        into tensor i's gradient buffer on the library's copy stream, and the
+        step of each group of tensors starts as soon as that group's copies are
+        done.  ``amax_out`` (CPU float32 [2 * T], pinned) receives amax_m then
+        amax_v.  Asynchronous: keep the host tensors alive and read
+        ``amax_out`` only after ``stream`` has been synchronised."""
+        if len(host_grads) != len(self.params):
+            raise ValueError("one host gradient per tensor")
+        ptrs = (ctypes.c_void_p * len(host_grads))()
+        for i, (h, p) in enumerate(zip(host_grads, self.params)):
+            if h.device.type != "cpu" or h.dtype != torch.bfloat16 or h.numel() != p.numel() or \
+                    not h.is_contiguous():
+                raise ValueError("host gradient %d: contiguous CPU bf16 of %d elements expected" % (i, p.numel()))
+            ptrs[i] = h.data_ptr() if h.numel() else None
+        out = 0
+        if amax_out is not None:
+            if amax_out.device.type != "cpu" or amax_out.dtype != torch.float32 or \
+                    amax_out.numel() != 2 * len(self.params) or not amax_out.is_contiguous():
+                raise ValueError("amax_out: contiguous CPU float32 of 2 * T elements expected")
+            out = amax_out.data_ptr()
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        self.t += 1
+        lr = self.lr if lr is None else lr
+        sp = capi.fp8adam_step_params(lr, self.betas[0], self.betas[1], self.eps, self.weight_decay, self.t,
+                                      loss_scale, max_norm, 1 if skip_nonfinite else 0)
+        try:
+            capi.fp8adam_step_host(self.ctx, sp, ptrs, out, s.cuda_stream)
+        except capi.Fp8AdamError:
+            self.t -= 1
+            raise
+
     def grad_info(self, stream: Optional[torch.cuda.Stream] = None):
         """(global grad L2 norm, skipped) of the last step with a gradient
         pre-pass (synchronises the stream)."""

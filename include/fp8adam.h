@@ -210,6 +210,30 @@ typedef struct {
 int fp8adam_step_ex(fp8adam_ctx* ctx, const fp8adam_step_params* params,
                     void* cuda_stream);
 
+/* One step (as fp8adam_step_ex) whose gradients come from host memory.
+ * host_grads: host array [num_tensors] of host pointers; host_grads[i] holds
+ * tensor i's numel bf16 gradients (may be NULL for an empty tensor).  Pinned
+ * (page-locked) buffers let the copies run asynchronously and overlap the
+ * step.  Each is copied into the tensor's device gradient buffer (the grad
+ * pointer given at create) on a copy stream owned by the context, which first
+ * waits for the work already queued on cuda_stream.  The tensors are taken in
+ * up to 8 groups of about equal size, cut at tensor boundaries; the step of a
+ * group is queued on cuda_stream behind that group's copies only, so the
+ * copies of later groups overlap it.  With loss_scale != 1, max_norm > 0 or
+ * skip_nonfinite the step waits for all copies (the global norm needs every
+ * gradient).  amax_host (optional, host float [2 * num_tensors], pinned for
+ * an asynchronous copy): receives amax_m then amax_v of this step.
+ * Asynchronous: host buffers must stay valid, and amax_host is written, only
+ * once the work queued on cuda_stream has completed.  The results equal
+ * fp8adam_step_ex after copying the gradients.  Returns INVALID_ARG for a
+ * NULL host pointer of a non-empty tensor or bad parameters, WRONG_DEVICE,
+ * CUDA on a failed copy or launch.
+ * Source of the step: as fp8adam_step_ex; the host-to-device gradient copy
+ * is this library's end-to-end entry point (no passage on the pages). */
+int fp8adam_step_host(fp8adam_ctx* ctx, const fp8adam_step_params* params,
+                      const uint16_t* const* host_grads, float* amax_host,
+                      void* cuda_stream);
+
 /* Results of the last fp8adam_step_ex pre-pass: *grad_norm = the global L2
  * norm of the unscaled gradients, *skipped = 1 if that step was skipped.
  * Host outputs; waits for cuda_stream.  Zeros if no pre-pass ran. */

@@ -29,7 +29,7 @@ class Run:
     def __init__(self, specs, cfg_id: int, m_fmt: int = oracle.E4M3, v_fmt: int = oracle.E5M2,
                  subset: Optional[Sequence[int]] = None, stats: bool = False,
                  jit_every_step: bool = False, hp: Optional[dict] = None,
-                 model: Optional[workloads.FlatModel] = None, init: bool = True):
+                 model: Optional[workloads.FlatModel] = None, init: bool = True, host: bool = False):
         self.specs, self.cfg_id = specs, cfg_id
         self.m_fmt, self.v_fmt = m_fmt, v_fmt
         self.hp = dict(HP if hp is None else hp)
@@ -47,6 +47,13 @@ class Run:
                             lr=self.hp["lr"], betas=(self.hp["beta1"], self.hp["beta2"]),
                             eps=self.hp["eps"], weight_decay=self.hp["weight_decay"])
         self.subset = list(range(len(specs))) if subset is None else list(subset)
+        # host mode: gradients reach the library from pinned host memory
+        # through fp8adam_step_host; the device buffer is zeroed first, so
+        # only the library's own copy can supply them
+        self.host = host
+        if host:
+            self.g_host = torch.empty(M.g.numel(), dtype=torch.bfloat16, pin_memory=True)
+            self.amax_host = torch.zeros(2 * len(specs), dtype=torch.float32, pin_memory=True)
         torch.cuda.synchronize()
         self.ref: Dict[int, oracle.TensorState] = {
             i: oracle.TensorState(M.view(M.p, i).cpu().numpy(), m_fmt, v_fmt) for i in self.subset}
@@ -59,7 +66,16 @@ class Run:
     def step(self, with_oracle: bool = True) -> None:
         self.t += 1
         self.draw_grads(self.t)
-        self.opt.step()
+        if self.host:
+            M = self.model
+            self.g_host.copy_(M.g)
+            M.g.zero_()
+            views = [self.g_host[o:o + s.numel] for o, s in zip(M.off, self.specs)]
+            self.opt.step_host(views, self.amax_host)
+            torch.cuda.synchronize()
+            M.g.copy_(self.g_host)  # what the oracle reads
+        else:
+            self.opt.step()
         if with_oracle:
             self.oracle_step()
 

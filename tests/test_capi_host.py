@@ -87,6 +87,13 @@ def test_binding_raises_on_error_codes(L):
     assert e.value.code == capi.ERR_INVALID_ARG
 
 
+def test_host_step_rejects_bad_arguments_on_host(L):
+    sp = capi.fp8adam_step_params(1e-3, 0.9, 0.95, 1e-8, 0.1, 1, 1.0, 0.0, 0)
+    ptrs = (ctypes.c_void_p * 1)()
+    assert L.fp8adam_step_host(None, ctypes.byref(sp), ptrs, None, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_step_host(None, None, ptrs, None, None) == capi.ERR_INVALID_ARG
+
+
 def test_option_entry_points_reject_bad_arguments_on_host(L):
     T = capi.fp8adam_tensor * 1
     t = T(capi.fp8adam_tensor(8, 8, 8, 8, 16))

@@ -198,3 +198,25 @@ def test_options_on_misaligned_views():
         assert (m[i].cpu().numpy() == rs.m).all() and (v[i].cpu().numpy() == rs.v).all(), i
         assert (p[i].cpu().numpy().view(np.uint32) == rs.p.view(np.uint32)).all(), i
         assert (pb[i].cpu().view(torch.int16).numpy().view(np.uint16) == rs.p_bf16).all(), i
+
+
+def test_options_through_host_step():
+    """fp8adam_step_host with options: the history and stochastic rounding
+    (grouped steps), then loss scale and clipping (one group after all
+    copies); the same results as copying the gradients and fp8adam_step_ex."""
+    a = ExtRun(50, amax_history_len=3, stochastic_rounding=True, seed=7)
+    b = ExtRun(50, amax_history_len=3, stochastic_rounding=True, seed=7)
+    h = torch.empty(b.M.g.numel(), dtype=torch.bfloat16, pin_memory=True)
+    views = [h[o:o + s.numel] for o, s in zip(b.M.off, b.specs)]
+    for t in range(1, 6):
+        kw = dict(loss_scale=64.0, max_norm=0.5) if t >= 4 else {}
+        a.step(**kw)
+        workloads.grads_into(b.specs, b.M.views(b.M.g), b.cfg, t, b.sig)
+        h.copy_(b.M.g)
+        b.M.g.zero_()
+        b.opt.step_host(views, **kw)
+        torch.cuda.synchronize()
+        for x in ("p", "m", "v", "scale_m", "scale_v", "amax_m", "amax_v"):
+            assert torch.equal(getattr(a.M, x).view(torch.uint8), getattr(b.M, x).view(torch.uint8)), (t, x)
+        assert torch.equal(a.opt.hist_m, b.opt.hist_m)
+    a.compare()  # and a against the oracle

@@ -288,3 +288,20 @@ def test_llama2_7b_layout_subset_3_steps():
         r.step()
         r.compare()
         r.check_invariants()
+
+
+@pytest.mark.parametrize("jit", [False, True], ids=["delayed", "jit_every_step"])
+def test_step_from_host_buffers(jit):
+    """fp8adam_step_host: gradients copied from pinned host memory by the
+    library (the device buffer is zeroed before each step), the step of each
+    tensor group overlapping the copies of the next groups; every element
+    against the oracle, and the amax read back to the host."""
+    sizes = [70001, 0, 4096, 33, 3 * 65536 + 4099, 17, 200003, 1, 131072, 65535, 9000, 4097]
+    specs = workloads.custom_layout(sizes)
+    r = Run(specs, 14, host=True, jit_every_step=jit)
+    for _ in range(4):
+        r.step()
+        r.compare()
+        M = r.model
+        assert torch.equal(r.amax_host[:len(specs)], M.amax_m.cpu()) and \
+            torch.equal(r.amax_host[len(specs):], M.amax_v.cpu())
