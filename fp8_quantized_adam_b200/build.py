@@ -13,8 +13,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfp8adam.so")
+LIB_DEBUG = os.path.join(PKG, "libfp8adam_debug.so")  # bounds checks, wait injection (FP8ADAM_DEBUG)
 SOURCES = [os.path.join(CSRC, "fp8adam_capi.cu"), os.path.join(CSRC, "fp8adam_noalloc.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fp8_codec.cuh", "fp8adam_step.cuh", "fp8adam_ext.cuh", "fp8adam_step_tma.cuh", "fp8adam_ext_tma.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fp8_codec.cuh", "fp8adam_step.cuh", "fp8adam_ext.cuh", "fp8adam_step_tma.cuh", "fp8adam_ext_tma.cuh", "fp8adam_debug.cuh")] + [
     os.path.join(ROOT, "include", "fp8adam.h")]
 
 NVCC_FLAGS = [
@@ -33,17 +34,27 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+def _build_one(lib: str, flags, force: bool, verbose: bool) -> str:
     newest = max(os.path.getmtime(p) for p in DEPS)
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest and not extra:
-        return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-o", tmp, *SOURCES]
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= newest:
+        return lib
+    tmp = lib + ".tmp%d" % os.getpid()
+    cmd = [nvcc(), *NVCC_FLAGS, *flags, "-o", tmp, *SOURCES]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False, extra=(), debug: bool = True) -> str:
+    """The release library (returned) and, unless debug=False, the debug one."""
+    if extra:
+        force = True
+    lib = _build_one(LIB, list(extra), force, verbose)
+    if debug:
+        _build_one(LIB_DEBUG, ["-DFP8ADAM_DEBUG", *extra], force, verbose)
+    return lib
 
 
 if __name__ == "__main__":

@@ -11,6 +11,7 @@ import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfp8adam.so")
+DEBUG_LIB_PATH = os.path.join(_PKG, "libfp8adam_debug.so")
 
 OK = 0
 ERR_INVALID_ARG = -1
@@ -20,6 +21,7 @@ ERR_OOM = -4
 ERR_WRONG_DEVICE = -5
 ERR_NOALLOC_LIMIT = -6
 ERR_DEVICE_TIMEOUT = -7
+ERR_DEBUG_BOUNDS = -8
 NOALLOC_MAX_TENSORS = 4096
 
 E4M3, E5M2, FP32 = 0, 1, 2
@@ -57,6 +59,7 @@ class Fp8AdamError(RuntimeError):
 
 
 _lib = None
+_debug_lib = None
 
 
 def lib() -> ctypes.CDLL:
@@ -65,48 +68,67 @@ def lib() -> ctypes.CDLL:
     if _lib is None:
         if not os.path.exists(LIB_PATH):
             raise RuntimeError("libfp8adam.so is not built (python -m fp8_quantized_adam_b200.build)")
-        L = ctypes.CDLL(LIB_PATH)
-        vp, i32, i64, u32, f = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float
-        L.fp8adam_create.restype = ctypes.c_int
-        L.fp8adam_create.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, vp, vp, vp, vp, i32, i32, u32,
-                                     ctypes.POINTER(vp)]
-        L.fp8adam_step.restype = ctypes.c_int
-        L.fp8adam_step.argtypes = [vp, f, f, f, f, f, i64, vp]
-        L.fp8adam_get_stats.restype = ctypes.c_int
-        L.fp8adam_get_stats.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), vp]
-        L.fp8adam_reset_stats.restype = ctypes.c_int
-        L.fp8adam_reset_stats.argtypes = [vp, vp]
-        L.fp8adam_destroy.restype = ctypes.c_int
-        L.fp8adam_destroy.argtypes = [vp]
-        L.fp8adam_strerror.restype = ctypes.c_char_p
-        L.fp8adam_strerror.argtypes = [ctypes.c_int]
-        L.fp8adam_encode.restype = ctypes.c_int
-        L.fp8adam_encode.argtypes = [i32, vp, vp, i64, i32, vp]
-        L.fp8adam_encode_bits_range.restype = ctypes.c_int
-        L.fp8adam_encode_bits_range.argtypes = [i32, u32, i64, vp, i32, vp]
-        L.fp8adam_decode.restype = ctypes.c_int
-        L.fp8adam_decode.argtypes = [i32, vp, vp, i64, i32, vp]
-        L.fp8adam_step_host.restype = ctypes.c_int
-        L.fp8adam_step_host.argtypes = [vp, ctypes.POINTER(fp8adam_step_params), ctypes.POINTER(ctypes.c_void_p),
-                                        vp, vp]
-        L.fp8adam_encode_sr.restype = ctypes.c_int
-        L.fp8adam_encode_sr.argtypes = [i32, vp, vp, vp, i64, vp]
-        L.fp8adam_launch_count.restype = ctypes.c_uint64
-        L.fp8adam_launch_count.argtypes = []
-        L.fp8adam_create_ex.restype = ctypes.c_int
-        L.fp8adam_create_ex.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, ctypes.POINTER(fp8adam_options),
-                                        ctypes.POINTER(vp)]
-        L.fp8adam_step_ex.restype = ctypes.c_int
-        L.fp8adam_step_ex.argtypes = [vp, ctypes.POINTER(fp8adam_step_params), vp]
-        L.fp8adam_check.restype = ctypes.c_int
-        L.fp8adam_check.argtypes = [vp, vp]
-        L.fp8adam_get_grad_info.restype = ctypes.c_int
-        L.fp8adam_get_grad_info.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint32), vp]
-        L.fp8adam_step_noalloc.restype = ctypes.c_int
-        L.fp8adam_step_noalloc.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, vp, vp, vp, vp, i32, i32, u32,
-                                           f, f, f, f, f, i64, vp]
-        _lib = L
+        _lib = _bind(ctypes.CDLL(LIB_PATH))
     return _lib
+
+
+def debug_lib() -> ctypes.CDLL:
+    """The debug build (bounds checks that report FP8ADAM_ERR_DEBUG_BOUNDS,
+    the bounded-wait injection point), same C ABI; for tests."""
+    global _debug_lib
+    if _debug_lib is None:
+        if not os.path.exists(DEBUG_LIB_PATH):
+            raise RuntimeError("libfp8adam_debug.so is not built (python -m fp8_quantized_adam_b200.build)")
+        _debug_lib = _bind(ctypes.CDLL(DEBUG_LIB_PATH))
+    return _debug_lib
+
+
+def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
+    """Argument and result types of every exported call."""
+    vp, i32, i64, u32, f = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float
+    L.fp8adam_create.restype = ctypes.c_int
+    L.fp8adam_create.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, vp, vp, vp, vp, i32, i32, u32,
+                                 ctypes.POINTER(vp)]
+    L.fp8adam_step.restype = ctypes.c_int
+    L.fp8adam_step.argtypes = [vp, f, f, f, f, f, i64, vp]
+    L.fp8adam_get_stats.restype = ctypes.c_int
+    L.fp8adam_get_stats.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), vp]
+    L.fp8adam_reset_stats.restype = ctypes.c_int
+    L.fp8adam_reset_stats.argtypes = [vp, vp]
+    L.fp8adam_destroy.restype = ctypes.c_int
+    L.fp8adam_destroy.argtypes = [vp]
+    L.fp8adam_strerror.restype = ctypes.c_char_p
+    L.fp8adam_strerror.argtypes = [ctypes.c_int]
+    L.fp8adam_encode.restype = ctypes.c_int
+    L.fp8adam_encode.argtypes = [i32, vp, vp, i64, i32, vp]
+    L.fp8adam_encode_bits_range.restype = ctypes.c_int
+    L.fp8adam_encode_bits_range.argtypes = [i32, u32, i64, vp, i32, vp]
+    L.fp8adam_decode.restype = ctypes.c_int
+    L.fp8adam_decode.argtypes = [i32, vp, vp, i64, i32, vp]
+    L.fp8adam_step_host.restype = ctypes.c_int
+    L.fp8adam_step_host.argtypes = [vp, ctypes.POINTER(fp8adam_step_params), ctypes.POINTER(ctypes.c_void_p),
+                                    vp, vp]
+    L.fp8adam_encode_sr.restype = ctypes.c_int
+    L.fp8adam_encode_sr.argtypes = [i32, vp, vp, vp, i64, vp]
+    L.fp8adam_launch_count.restype = ctypes.c_uint64
+    L.fp8adam_launch_count.argtypes = []
+    L.fp8adam_create_ex.restype = ctypes.c_int
+    L.fp8adam_create_ex.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, ctypes.POINTER(fp8adam_options),
+                                    ctypes.POINTER(vp)]
+    L.fp8adam_step_ex.restype = ctypes.c_int
+    L.fp8adam_step_ex.argtypes = [vp, ctypes.POINTER(fp8adam_step_params), vp]
+    L.fp8adam_check.restype = ctypes.c_int
+    L.fp8adam_check.argtypes = [vp, vp]
+    L.fp8adam_get_grad_info.restype = ctypes.c_int
+    L.fp8adam_get_grad_info.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint32), vp]
+    L.fp8adam_step_noalloc.restype = ctypes.c_int
+    L.fp8adam_step_noalloc.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, vp, vp, vp, vp, i32, i32, u32,
+                                       f, f, f, f, f, i64, vp]
+    L.fp8adam_debug_inject_wait.restype = ctypes.c_int
+    L.fp8adam_debug_inject_wait.argtypes = [i32, i32]
+    L.fp8adam_debug_set_numel.restype = ctypes.c_int
+    L.fp8adam_debug_set_numel.argtypes = [vp, i32, i64]
+    return L
 
 
 def _check(fn: str, rc: int) -> int:
@@ -209,4 +231,5 @@ def fp8adam_step_noalloc(tensors, num_tensors: int, scale_m: int, scale_v: int, 
 EXPORTED = ["fp8adam_create", "fp8adam_step", "fp8adam_get_stats", "fp8adam_reset_stats",
             "fp8adam_destroy", "fp8adam_strerror", "fp8adam_encode", "fp8adam_encode_bits_range",
             "fp8adam_decode", "fp8adam_launch_count", "fp8adam_step_noalloc", "fp8adam_create_ex",
-            "fp8adam_step_ex", "fp8adam_get_grad_info", "fp8adam_check", "fp8adam_encode_sr", "fp8adam_step_host"]
+            "fp8adam_step_ex", "fp8adam_get_grad_info", "fp8adam_check", "fp8adam_encode_sr", "fp8adam_step_host",
+            "fp8adam_debug_inject_wait", "fp8adam_debug_set_numel"]

@@ -7,8 +7,10 @@
 // The kernels are in fp8adam_step.cuh; the codec in fp8_codec.cuh.
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
+#include <cstddef>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -182,6 +184,14 @@ ExtFn pick_amax_ext(int mf, int vf) {
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// NVTX range over a host call (visible to Nsight tools; a no-op without one)
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 }  // namespace
 
@@ -528,6 +538,7 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
   e.skip = nullptr;
   e.p_bf16 = ctx->d_bf16;
   if (prepass) {
+    NvtxRange pre("fp8adam grad-norm pre-pass");
     if (cudaMemsetAsync(ctx->d_nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)
       return FP8ADAM_ERR_CUDA;
     fp8adam_gradnorm_partial_kernel<<<grid, block, 0, st>>>(a, ctx->d_partial, ctx->d_nonfinite);
@@ -565,6 +576,7 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
 }
 
 static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t st) {
+  NvtxRange range("fp8adam_step");
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return FP8ADAM_ERR_CUDA;
   if (dev != ctx->device) return FP8ADAM_ERR_WRONG_DEVICE;
@@ -635,6 +647,7 @@ extern "C" int fp8adam_step_host(fp8adam_ctx* ctx, const fp8adam_step_params* pa
   // one group; otherwise group g's step waits only for group g's copies
   const bool whole = needs_prepass(p);
   const int ng = whole ? 1 : G;
+  NvtxRange range("fp8adam_step_host");
   for (int g = 0; g < ng; ++g) {
     const int32_t t0 = whole ? 0 : ctx->grp_tensor[(size_t)g];
     const int32_t t1 = whole ? ctx->T : ctx->grp_tensor[(size_t)g + 1];
@@ -698,11 +711,58 @@ extern "C" int fp8adam_reset_stats(fp8adam_ctx* ctx, void* cuda_stream) {
 extern "C" int fp8adam_check(fp8adam_ctx* ctx, void* cuda_stream) {
   if (!ctx) return FP8ADAM_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  uint32_t e = 0;
-  if (cudaMemcpyAsync(&e, ctx->d_error, sizeof(e), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
+  uint32_t e = 0, bounds = 0;
+  if (cudaMemcpyAsync(&e, ctx->d_error, sizeof(e), cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return FP8ADAM_ERR_CUDA;
-  return e ? FP8ADAM_ERR_DEVICE_TIMEOUT : FP8ADAM_OK;
+#ifdef FP8ADAM_DEBUG
+  if (cudaMemcpyFromSymbolAsync(&bounds, g_debug_flags, sizeof(bounds), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return FP8ADAM_ERR_CUDA;
+#endif
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
+  if (!e && !bounds) return FP8ADAM_OK;
+  // A step stopped part-way: clear the error word and the per-step device
+  // state (amax accumulators, JIT amax, chunk counters) so the next step
+  // starts clean.  The elements of the failed step are partly updated.
+  const uint32_t zero = 0;
+  if (cudaMemsetAsync(ctx->d_state, 0, 5 * (size_t)ctx->T * sizeof(uint32_t), st) != cudaSuccess ||
+      cudaMemsetAsync(ctx->d_error, 0, sizeof(uint32_t), st) != cudaSuccess)
+    return FP8ADAM_ERR_CUDA;
+#ifdef FP8ADAM_DEBUG
+  if (cudaMemcpyToSymbolAsync(g_debug_flags, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return FP8ADAM_ERR_CUDA;
+#endif
+  (void)zero;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
+  return bounds ? FP8ADAM_ERR_DEBUG_BOUNDS : FP8ADAM_ERR_DEVICE_TIMEOUT;
+}
+
+extern "C" int fp8adam_debug_inject_wait(int32_t cta, int32_t subtile) {
+#ifdef FP8ADAM_DEBUG
+  if (cudaMemcpyToSymbol(g_inject_cta, &cta, sizeof(cta)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_inject_sub, &subtile, sizeof(subtile)) != cudaSuccess)
+    return FP8ADAM_ERR_CUDA;
+  return FP8ADAM_OK;
+#else
+  (void)cta;
+  (void)subtile;
+  return FP8ADAM_ERR_INVALID_ARG;  // the release build has no injection point
+#endif
+}
+
+extern "C" int fp8adam_debug_set_numel(fp8adam_ctx* ctx, int32_t tensor, int64_t numel) {
+#ifdef FP8ADAM_DEBUG
+  if (!ctx || tensor < 0 || tensor >= ctx->T || numel < 0 || numel > ctx->numel[(size_t)tensor])
+    return FP8ADAM_ERR_INVALID_ARG;
+  if (cudaMemcpy(reinterpret_cast<char*>(ctx->d_tensors + tensor) + offsetof(TensorDesc, numel), &numel,
+                 sizeof(numel), cudaMemcpyHostToDevice) != cudaSuccess)
+    return FP8ADAM_ERR_CUDA;
+  return FP8ADAM_OK;
+#else
+  (void)ctx;
+  (void)tensor;
+  (void)numel;
+  return FP8ADAM_ERR_INVALID_ARG;
+#endif
 }
 
 extern "C" int fp8adam_destroy(fp8adam_ctx* ctx) {
@@ -718,6 +778,7 @@ extern "C" const char* fp8adam_strerror(int code) {
     case FP8ADAM_ERR_INVALID_ARG: return "invalid argument";
     case FP8ADAM_ERR_UNSUPPORTED_FMT: return "unsupported moment format";
     case FP8ADAM_ERR_CUDA: return "CUDA runtime error";
+    case FP8ADAM_ERR_DEBUG_BOUNDS: return "a kernel access outside its tensor was skipped (debug build)";
     case FP8ADAM_ERR_OOM: return "device allocation failed";
     case FP8ADAM_ERR_WRONG_DEVICE: return "current device differs from the context's";
     case FP8ADAM_ERR_NOALLOC_LIMIT: return "more tensors than the allocation-free step holds (FP8ADAM_NOALLOC_MAX_TENSORS)";

@@ -182,6 +182,7 @@ struct ExtSeg {  // per tensor segment
 template <int MF, int VF, bool STATS, int SRM>
 __device__ __forceinline__ void ext_element(const ExtArgs& a, const TensorDesc& td, const ExtSeg& sg, int64_t i,
                                             float& am, float& av, uint32_t& flushed, uint32_t& sat) {
+  FP8ADAM_BOUNDS(i >= 0 && i < td.numel);
   const StepConsts& c = a.s.c;
   uint32_t rm = 0, rv = 0;
   if (use_sr<SRM>(a)) {
@@ -208,6 +209,7 @@ __device__ __forceinline__ void ext_element(const ExtArgs& a, const TensorDesc& 
 template <int MF, int VF, bool STATS, int SRM>
 __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& td, const ExtSeg& sg, int64_t i,
                                             float& am, float& av, uint32_t& flushed, uint32_t& sat) {
+  FP8ADAM_BOUNDS(i >= 0 && i + kVec <= td.numel);
   const StepConsts& c = a.s.c;
   float4 pv[4];
 #pragma unroll
@@ -369,7 +371,9 @@ fp8adam_step_ext_kernel(const ExtArgs a) {
   const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
   const Chunk ch = a.s.chunks[blockIdx.x];
   const int ti = ch.tensor;
+  FP8ADAM_BOUNDS(ti >= 0 && ti < a.s.num_tensors);
   const TensorDesc td = a.s.tensors[ti];
+  FP8ADAM_BOUNDS(ch.start >= 0 && ch.len >= 0 && ch.start + ch.len <= td.numel);
   const ExtSeg sg = ext_setup<MF, VF>(a, ti, gm);
   float am = 0.0f, av = 0.0f;
   uint32_t flushed = 0, sat = 0;
@@ -390,8 +394,10 @@ fp8adam_amax_ext_kernel(const ExtArgs a) {
   const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
   const Chunk ch = S.chunks[blockIdx.x];
   const int ti = ch.tensor;
+  FP8ADAM_BOUNDS(ti >= 0 && ti < S.num_tensors);
   const TensorDesc td = S.tensors[ti];
   const int64_t e0 = ch.start, e1 = ch.start + ch.len;
+  FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
   const float inv_s_m = __fdiv_rn(1.0f, S.scale_m[ti]);
   const float inv_s_v = __fdiv_rn(1.0f, S.scale_v[ti]);
   float am = 0.0f, av = 0.0f;
@@ -483,8 +489,10 @@ fp8adam_gradnorm_partial_kernel(const StepArgs a, double* partial, unsigned long
   double acc = 0.0;
   uint32_t bad = 0;
   const Chunk ch = a.chunks[blockIdx.x];
+  FP8ADAM_BOUNDS(ch.tensor >= 0 && ch.tensor < a.num_tensors);
   const TensorDesc td = a.tensors[ch.tensor];
   const int64_t e0 = ch.start, e1 = ch.start + ch.len;
+  FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
   int64_t scalar_from = e0;
   if (td.aligned) {
     for (int64_t i = e0 + (int64_t)threadIdx.x * kVec; i + kVec <= e1; i += kTile) {

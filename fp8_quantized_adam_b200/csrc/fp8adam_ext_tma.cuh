@@ -43,6 +43,7 @@ template <int MF, int VF, bool STATS, bool SR>
 __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& st, int j, const TensorDesc& td,
                                              const ExtSeg& sg, const SrChunk& su, int64_t i, float& am, float& av,
                                              uint32_t& flushed, uint32_t& sat) {
+  FP8ADAM_BOUNDS(i >= 0 && i + 4 <= td.numel);
   const StepConsts& c = a.s.c;
   const float4 pin = *reinterpret_cast<const float4*>(&st.p[j]);
   const uint2 gq = *reinterpret_cast<const uint2*>(&st.g[j]);
@@ -127,9 +128,11 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
   const Chunk ch = a.s.chunks[blockIdx.x];
   const int ti = ch.tensor;
+  FP8ADAM_BOUNDS(ti >= 0 && ti < a.s.num_tensors);
   const TensorDesc td = a.s.tensors[ti];
   const ExtSeg sg = ext_setup<MF, VF>(a, ti, gm);
   const int64_t e0 = ch.start, e1 = ch.start + ch.len;
+  FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
   float am = 0.0f, av = 0.0f;
   uint32_t flushed = 0, sat = 0;
 

@@ -26,6 +26,7 @@
 #include <stdint.h>
 
 #include "fp8_codec.cuh"
+#include "fp8adam_debug.cuh"
 
 namespace fp8adam {
 
@@ -255,6 +256,7 @@ template <int MF, int VF, bool STATS, bool WRITE>
 __device__ __forceinline__ void group16(const TensorDesc& td, int64_t i, const StepConsts& c, float inv_s_m,
                                         float inv_s_v, float s_m_new, float s_v_new, float& am, float& av,
                                         uint32_t& flushed, uint32_t& sat) {
+  FP8ADAM_BOUNDS(i >= 0 && i + kVec <= td.numel);
   float4 pv[4];
   if constexpr (WRITE) {
 #pragma unroll
@@ -301,6 +303,7 @@ template <int MF, int VF, bool STATS, bool WRITE>
 __device__ __forceinline__ void element1(const TensorDesc& td, int64_t i, const StepConsts& c, float inv_s_m,
                                          float inv_s_v, float s_m_new, float s_v_new, float& am, float& av,
                                          uint32_t& flushed, uint32_t& sat) {
+  FP8ADAM_BOUNDS(i >= 0 && i < td.numel);
   const float g = __uint_as_float((uint32_t)td.g[i] << 16);
   float mn, vn;
   moments(c, g, load1<MF>(td.m, i, inv_s_m), load1<VF>(td.v, i, inv_s_v), mn, vn);
@@ -322,7 +325,9 @@ __device__ __forceinline__ void element1(const TensorDesc& td, int64_t i, const 
 template <int MF, int VF, bool STATS, bool WRITE>
 __device__ __forceinline__ void run_segment(const StepArgs& a, int ti, int64_t e0, int64_t e1, uint32_t units,
                                             uint32_t (*red)[kThreads / 32]) {
+  FP8ADAM_BOUNDS(ti >= 0 && ti < a.num_tensors);
   const TensorDesc td = a.tensors[ti];
+  FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
   const StepConsts c = a.c;
   const float s_m = a.scale_m[ti];
   const float s_v = a.scale_v[ti];

@@ -17,7 +17,8 @@
 //
 // A tensor that is not 16-byte aligned, and the part of a chunk beyond its
 // last whole sub-tile, go through the per-thread path of fp8adam_step.cuh.
-// Every wait is bounded: on a timeout the CTA sets bit 0 of *err, waits
+// Every wait is bounded in time (about 1 s on the global timer, each try
+// suspending at most 20 us): on a timeout the CTA sets bit 0 of *err, waits
 // (bounded) for its copies in flight and leaves the chunk unfinished; CTAs
 // that start later see the flag and return at once (the host reads it
 // through fp8adam_check).
@@ -32,7 +33,11 @@ namespace fp8adam {
 
 constexpr int kSub = 2048;                    // elements per stage (2 x 4 per thread)
 constexpr int kStages = 3;
-constexpr uint32_t kWaitLimit = 1u << 22;     // try_wait polls before giving up
+// Bounded waits: each try suspends at most kSuspendNs (the hint); a wait
+// gives up after kWaitNs on the global timer, or after kWaitLimit tries.
+constexpr uint32_t kSuspendNs = 20000;        // 20 us
+constexpr uint32_t kWaitNs = 1000000000u;     // 1 s (the timer's low word wraps after 4.29 s)
+constexpr uint32_t kWaitLimit = 1u << 20;
 
 struct __align__(128) TmaStage {              // 16 KB
   float p[kSub];
@@ -55,16 +60,25 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
-// bounded wait; false if the limit ran out
+__device__ __forceinline__ uint32_t globaltimer_lo_ns() {
+  uint32_t t;
+  asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
+  return t;
+}
+// bounded wait; false if the limit ran out.  The first try needs no timer.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kWaitLimit; ++it)
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t t0 = globaltimer_lo_ns();
+  for (uint32_t it = 0; it < kWaitLimit; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_lo_ns() - t0 > kWaitNs) return false;  // modular: exact across a wrap
+  }
   return false;
 }
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`
@@ -83,6 +97,7 @@ template <int MF, int VF, bool STATS>
 __device__ __forceinline__ void consume4(const TmaStage& st, int j, const TensorDesc& td, int64_t i,
                                          const StepConsts& c, float inv_s_m, float inv_s_v, float s_m_new,
                                          float s_v_new, float& am, float& av, uint32_t& flushed, uint32_t& sat) {
+  FP8ADAM_BOUNDS(i >= 0 && i + 4 <= td.numel);
   const float4 pin = *reinterpret_cast<const float4*>(&st.p[j]);
   const uint2 gq = *reinterpret_cast<const uint2*>(&st.g[j]);
   const uint32_t mw = *reinterpret_cast<const uint32_t*>(&st.m[j]);
@@ -141,6 +156,7 @@ __device__ __forceinline__ bool tma_stream(const TensorDesc& td, int64_t e0, int
     uint64_t* bar = &full[k % kStages];
     const int64_t b = e0 + (int64_t)k * kSub;
     mbar_arrive_expect_tx(bar, (uint32_t)sizeof(TmaStage));
+    if (debug_skip_copies(k)) return;  // debug build: this stage's bytes never arrive
     bulk_load(st.p, td.p + b, kSub * 4, bar);
     bulk_load(st.g, td.g + b, kSub * 2, bar);
     bulk_load(st.m, static_cast<const uint8_t*>(td.m) + b, kSub, bar);
@@ -188,9 +204,11 @@ fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
   if (*(volatile const uint32_t*)err) return;  // an earlier CTA timed out: stop at once
   const Chunk ch = a.chunks[blockIdx.x];
   const int ti = ch.tensor;
+  FP8ADAM_BOUNDS(ti >= 0 && ti < a.num_tensors);
   const TensorDesc td = a.tensors[ti];
   const StepConsts c = a.c;
   const int64_t e0 = ch.start, e1 = ch.start + ch.len;
+  FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
   const float s_m = a.scale_m[ti];
   const float s_v = a.scale_v[ti];
   const float s_m_new = pow2scale<MF>(__uint_as_float(a.amax_in_m[ti]), s_m);

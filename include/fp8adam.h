@@ -67,6 +67,7 @@ extern "C" {
 #define FP8ADAM_ERR_WRONG_DEVICE (-5)    /* current device differs from create's */
 #define FP8ADAM_ERR_NOALLOC_LIMIT (-6)   /* more tensors than fp8adam_step_noalloc holds */
 #define FP8ADAM_ERR_DEVICE_TIMEOUT (-7)  /* a kernel's bounded wait ran out (see fp8adam_check) */
+#define FP8ADAM_ERR_DEBUG_BOUNDS (-8)    /* debug build: an access outside its tensor was skipped */
 
 /* Storage format of a moment. */
 typedef enum {
@@ -131,10 +132,29 @@ int fp8adam_get_stats(fp8adam_ctx* ctx, uint64_t* out, void* cuda_stream);
 int fp8adam_reset_stats(fp8adam_ctx* ctx, void* cuda_stream);
 
 /* Checks the context's device error word (waits for cuda_stream): returns
- * FP8ADAM_OK, or FP8ADAM_ERR_DEVICE_TIMEOUT if a step kernel's bounded wait
- * for its shared-memory copies ran out (a chunk was then left unfinished and
- * the state is not usable).  Host-side only otherwise. */
+ * FP8ADAM_OK; FP8ADAM_ERR_DEVICE_TIMEOUT if a step kernel's bounded wait for
+ * its shared-memory copies ran out (each wait gives up after about 1 s; the
+ * CTA waits, bounded, for its copies in flight and leaves its chunk
+ * unfinished, and CTAs that start later return at once); in the debug build,
+ * FP8ADAM_ERR_DEBUG_BOUNDS if a bounds check skipped an access.  On an error
+ * it also clears the error word and the per-step device state (amax
+ * accumulators, chunk counters), so the context can run the next step; the
+ * params and moments of the failed step are partly updated and should be
+ * restored from a checkpoint. */
 int fp8adam_check(fp8adam_ctx* ctx, void* cuda_stream);
+
+/* Debug build only (libfp8adam_debug.so, compiled with FP8ADAM_DEBUG; the
+ * release build returns FP8ADAM_ERR_INVALID_ARG and checks nothing).
+ * fp8adam_debug_inject_wait: from the next launch on, CTA `cta` of a staged
+ * step kernel arms the barrier of its sub-tile `subtile` but issues no copies
+ * for it, so that wait runs out and the kernel takes its timeout path (for
+ * testing the bounded waits without a GPU fault); -1, -1 switches it off.
+ * fp8adam_debug_set_numel: lowers tensor `tensor`'s element count in the
+ * device tensor table (not below 0, not above its real size), so the chunk
+ * table runs past it and the bounds checks fire (every access stays inside
+ * the real buffers). */
+int fp8adam_debug_inject_wait(int32_t cta, int32_t subtile);
+int fp8adam_debug_set_numel(fp8adam_ctx* ctx, int32_t tensor, int64_t numel);
 
 /* Frees the context (synchronises the device first).  NULL is accepted. */
 int fp8adam_destroy(fp8adam_ctx* ctx);

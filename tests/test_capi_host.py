@@ -87,6 +87,19 @@ def test_binding_raises_on_error_codes(L):
     assert e.value.code == capi.ERR_INVALID_ARG
 
 
+def test_release_build_has_no_debug_hooks(L):
+    assert L.fp8adam_debug_inject_wait(0, 1) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_debug_set_numel(None, 0, 0) == capi.ERR_INVALID_ARG
+
+
+def test_debug_build_loads_and_exports_the_same_symbols(L):
+    D = capi.debug_lib()
+    for name in capi.EXPORTED:
+        assert hasattr(D, name), name
+    assert D.fp8adam_debug_set_numel(None, 0, 0) == capi.ERR_INVALID_ARG  # host-side check, no GPU
+    assert D.fp8adam_strerror(capi.ERR_DEBUG_BOUNDS).startswith(b"a kernel access")
+
+
 def test_host_step_rejects_bad_arguments_on_host(L):
     sp = capi.fp8adam_step_params(1e-3, 0.9, 0.95, 1e-8, 0.1, 1, 1.0, 0.0, 0)
     ptrs = (ctypes.c_void_p * 1)()
