@@ -22,6 +22,7 @@ ERR_WRONG_DEVICE = -5
 ERR_NOALLOC_LIMIT = -6
 ERR_DEVICE_TIMEOUT = -7
 ERR_DEBUG_BOUNDS = -8
+ERR_OVERLAP = -9
 NOALLOC_MAX_TENSORS = 4096
 
 E4M3, E5M2, FP32 = 0, 1, 2

@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstddef>
 #include <cmath>
@@ -185,6 +186,25 @@ ExtFn pick_amax_ext(int mf, int vf) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+// True if two of the byte ranges overlap and at least one of them is
+// written.  Sorted by start, a range overlaps an earlier one iff it starts
+// before the furthest end seen so far (of any range if it is written, of
+// the written ranges if it is only read).
+struct ByteRange {
+  uintptr_t begin, end;
+  bool written;
+};
+bool written_range_overlaps(std::vector<ByteRange>& r) {
+  std::sort(r.begin(), r.end(), [](const ByteRange& a, const ByteRange& b) { return a.begin < b.begin; });
+  uintptr_t end_all = 0, end_written = 0;
+  for (const ByteRange& x : r) {
+    if (x.begin < (x.written ? end_all : end_written)) return true;
+    end_all = end_all > x.end ? end_all : x.end;
+    if (x.written) end_written = end_written > x.end ? end_written : x.end;
+  }
+  return false;
+}
+
 // NVTX range over a host call (visible to Nsight tools; a no-op without one)
 struct NvtxRange {
   explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
@@ -300,6 +320,28 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
     const fp8adam_tensor& t = tensors[i];
     if (t.numel < 0) return FP8ADAM_ERR_INVALID_ARG;
     if (t.numel > 0 && (!t.param || !t.grad || !t.m || !t.v)) return FP8ADAM_ERR_INVALID_ARG;
+  }
+  // no written buffer (p, m, v, the bf16 copy) may overlap any other buffer
+  try {
+    std::vector<ByteRange> ranges;
+    ranges.reserve((size_t)num_tensors * 5);
+    const size_t mb = m_fmt == FP8ADAM_FP32 ? 4 : 1, vb = v_fmt == FP8ADAM_FP32 ? 4 : 1;
+    for (int32_t i = 0; i < num_tensors; ++i) {
+      const fp8adam_tensor& t = tensors[i];
+      if (t.numel == 0) continue;
+      const size_t n = (size_t)t.numel;
+      auto add = [&](const void* p, size_t bytes, bool w) {
+        ranges.push_back(ByteRange{(uintptr_t)p, (uintptr_t)p + bytes, w});
+      };
+      add(t.param, 4 * n, true);
+      add(t.grad, 2 * n, false);
+      add(t.m, mb * n, true);
+      add(t.v, vb * n, true);
+      if (opts->param_bf16 && opts->param_bf16[i]) add(opts->param_bf16[i], 2 * n, true);
+    }
+    if (written_range_overlaps(ranges)) return FP8ADAM_ERR_OVERLAP;
+  } catch (...) {
+    return FP8ADAM_ERR_OOM;
   }
   int dev = -1, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -779,6 +821,7 @@ extern "C" const char* fp8adam_strerror(int code) {
     case FP8ADAM_ERR_UNSUPPORTED_FMT: return "unsupported moment format";
     case FP8ADAM_ERR_CUDA: return "CUDA runtime error";
     case FP8ADAM_ERR_DEBUG_BOUNDS: return "a kernel access outside its tensor was skipped (debug build)";
+    case FP8ADAM_ERR_OVERLAP: return "a written buffer (param, m, v or bf16 copy) overlaps another buffer";
     case FP8ADAM_ERR_OOM: return "device allocation failed";
     case FP8ADAM_ERR_WRONG_DEVICE: return "current device differs from the context's";
     case FP8ADAM_ERR_NOALLOC_LIMIT: return "more tensors than the allocation-free step holds (FP8ADAM_NOALLOC_MAX_TENSORS)";

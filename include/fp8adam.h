@@ -68,6 +68,7 @@ extern "C" {
 #define FP8ADAM_ERR_NOALLOC_LIMIT (-6)   /* more tensors than fp8adam_step_noalloc holds */
 #define FP8ADAM_ERR_DEVICE_TIMEOUT (-7)  /* a kernel's bounded wait ran out (see fp8adam_check) */
 #define FP8ADAM_ERR_DEBUG_BOUNDS (-8)    /* debug build: an access outside its tensor was skipped */
+#define FP8ADAM_ERR_OVERLAP (-9)         /* create: a written buffer overlaps another buffer */
 
 /* Storage format of a moment. */
 typedef enum {
@@ -105,7 +106,11 @@ typedef struct fp8adam_ctx fp8adam_ctx; /* opaque */
  * (host array) to the device, allocates the context's accumulators and
  * synchronises once.  scale_m/scale_v/amax_m/amax_v: device fp32
  * [num_tensors].  m_fmt/v_fmt: fp8adam_fmt.  Returns INVALID_ARG for null
- * pointers, num_tensors < 1 or numel < 0; UNSUPPORTED_FMT; OOM; CUDA. */
+ * pointers, num_tensors < 1 or numel < 0; UNSUPPORTED_FMT; OVERLAP if a
+ * buffer the step writes (param, m, v, and with fp8adam_create_ex the bf16
+ * copies) overlaps any other buffer of the list (gradients, which are only
+ * read, may overlap one another); OOM; CUDA.  Checked on the host before
+ * any CUDA call. */
 int fp8adam_create(const fp8adam_tensor* tensors, int32_t num_tensors,
                    float* scale_m, float* scale_v, float* amax_m,
                    float* amax_v, int32_t m_fmt, int32_t v_fmt,

@@ -87,6 +87,36 @@ def test_binding_raises_on_error_codes(L):
     assert e.value.code == capi.ERR_INVALID_ARG
 
 
+def test_create_rejects_overlapping_written_buffers_on_host(L):
+    """Checked before any CUDA call: fake addresses suffice.  A written buffer
+    (param, m, v) overlapping any other is OVERLAP; gradients may alias one
+    another; disjoint buffers get past the check (and then fail with CUDA on
+    a machine without a GPU, or succeed on one with a GPU)."""
+    T = capi.fp8adam_tensor
+    base = 1 << 32
+
+    def create(specs):
+        arr = (T * len(specs))(*[T(*x) for x in specs])
+        out = ctypes.c_void_p()
+        rc = L.fp8adam_create(arr, len(specs), 8, 8, 8, 8, 0, 1, 0, ctypes.byref(out))
+        if rc == capi.OK:  # a GPU is present: nothing was launched, just free the tables
+            L.fp8adam_destroy(out)
+        return rc
+
+    n = 1000
+    t0 = (base, base + 0x10000, base + 0x20000, base + 0x30000, n)
+    assert create([t0, t0]) == capi.ERR_OVERLAP                       # the same tensor twice
+    t1 = (base + 4 * n - 4, base + 0x40000, base + 0x50000, base + 0x60000, n)
+    assert create([t0, t1]) == capi.ERR_OVERLAP                       # params overlap by 4 bytes
+    t2 = (base + 0x70000, base + 0x10000, base + 0x80000, base + 0x90000, n)
+    assert create([t0, t2]) != capi.ERR_OVERLAP                       # shared gradient buffer: read only
+    t3 = (base + 0x70000, base + 0x80000, base + 0x90000, base + 0x10000 + 10, n)
+    assert create([t0, t3]) == capi.ERR_OVERLAP                       # a v written over a gradient
+    t4 = (base + 4 * n, base + 0xA0000, base + 0xB0000, base + 0xC0000, n)
+    assert create([t0, t4]) != capi.ERR_OVERLAP                       # adjacent, not overlapping
+    assert create([t0, (base, base, base, base, 0)]) != capi.ERR_OVERLAP  # an empty tensor has no bytes
+
+
 def test_release_build_has_no_debug_hooks(L):
     assert L.fp8adam_debug_inject_wait(0, 1) == capi.ERR_INVALID_ARG
     assert L.fp8adam_debug_set_numel(None, 0, 0) == capi.ERR_INVALID_ARG
