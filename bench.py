@@ -194,8 +194,9 @@ def reference_arm(args):
 
 def kernel_name(args) -> str:
     """The step kernel a run times (plus the norm pre-pass for clipping)."""
-    if args.variant == "default":
-        return "fp8adam_step_kernel<E4M3,E5M2>" if args.no_tma else "fp8adam_step_tma_kernel<E4M3,E5M2>"
+    if args.variant in ("default", "jit"):
+        k = "fp8adam_step_kernel<E4M3,E5M2>" if args.no_tma else "fp8adam_step_tma_kernel<E4M3,E5M2>"
+        return k + (" + amax pre-pass" if args.variant == "jit" else "")
     base = ("fp8adam_step_ext_kernel<E4M3,E5M2>" if args.no_tma else
             "fp8adam_step_ext_tma_kernel<E4M3,E5M2,SR=%d>" % (args.variant == "sr"))
     return base + (" + grad-norm pre-pass" if args.variant == "clip" else "")
@@ -242,6 +243,8 @@ def our_arm(args):
         opt_kw = dict(stochastic_rounding=True, seed=1234)
     elif args.variant == "history":
         opt_kw = dict(amax_history_len=16)
+    elif args.variant == "jit":
+        opt_kw = dict(jit_every_step=True)
     elif args.variant == "clip":
         step_kw = dict(loss_scale=1024.0, max_norm=1.0, skip_nonfinite=True)
     opt = FP8AdamW(model.views(model.p), model.views(model.g), m=model.views(model.m), v=model.views(model.v),
@@ -314,7 +317,8 @@ def our_arm(args):
     avg_kernel_s = sum(kernel_ms) / len(kernel_ms) / 1e3
     # bytes per param of one step: the fused clip/skip variant reads the
     # gradients once more in its norm pre-pass
-    bpp = BYTES_PER_PARAM + (2 if args.variant == "clip" else 0)
+    # and current scaling ("jit") runs an amax pre-pass over g, m, v first
+    bpp = BYTES_PER_PARAM + {"clip": 2, "jit": 4}.get(args.variant, 0)
     achieved = bpp * n_params / avg_kernel_s / 1e9
     traffic = None
     if TRAFFIC_PER_PARAM is not None and KERNEL_SHA == kernel_sha() and args.variant == "default" and not args.no_tma:
@@ -425,8 +429,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--chunk-elems", type=int, default=0, help="elements per CTA (0: chosen by the library)")
     ap.add_argument("--no-tma", action="store_true", help="per-thread vector loads instead of TMA staging")
-    ap.add_argument("--variant", choices=["default", "sr", "history", "clip"], default="default",
-                    help="step options: stochastic rounding, amax history 16, fused loss-scale/clip/skip")
+    ap.add_argument("--variant", choices=["default", "sr", "history", "clip", "jit"], default="default",
+                    help="step options: stochastic rounding, amax history 16, fused loss-scale/clip/skip, "
+                         "current scaling (amax pre-pass every step)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--report", choices=["ablation"], default=None,

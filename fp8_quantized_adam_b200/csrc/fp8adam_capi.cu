@@ -355,12 +355,13 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
     return n;
   };
   // chunk length: the largest that keeps >= 8 waves of resident CTAs (4 per
-  // SM), so the last partial wave costs little; never below 16384
+  // SM), so the last partial wave costs little; a list too small for that
+  // gets the shortest chunk (one 4096-element tile), for the most CTAs
   int64_t chunk = opts->chunk_elems;
   if (chunk == 0) {
     const int64_t want = (int64_t)sms * 4 * 8;
     chunk = kChunk;
-    while (chunk > 16384 && count_chunks(chunk) < want) chunk /= 2;
+    while (chunk > kTile && count_chunks(chunk) < want) chunk /= 2;
   }
   const int64_t total_units = count_chunks(chunk);
   if (total_units > INT32_MAX / 2) return FP8ADAM_ERR_INVALID_ARG;

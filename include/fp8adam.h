@@ -205,10 +205,10 @@ typedef struct {
                                   [numel] receiving the updated params rounded to
                                   nearest even (entries may be NULL), or NULL */
   int32_t chunk_elems;       /* elements per CTA: 0 = chosen from the list's size
-                                (the largest of 131072, 65536, 32768, 16384 giving
-                                at least 8 waves of CTAs); otherwise a multiple of
-                                4096 in [4096, 131072].  Results do not depend
-                                on it. */
+                                (the largest power of two in [4096, 131072]
+                                giving at least 8 waves of CTAs, else 4096);
+                                otherwise a multiple of 4096 in [4096, 131072].
+                                Results do not depend on it. */
 } fp8adam_options;
 
 /* fp8adam_create with options (fp8adam_create is this call with the options
