@@ -766,15 +766,14 @@ extern "C" int fp8adam_check(fp8adam_ctx* ctx, void* cuda_stream) {
   // A step stopped part-way: clear the error word and the per-step device
   // state (amax accumulators, JIT amax, chunk counters) so the next step
   // starts clean.  The elements of the failed step are partly updated.
-  const uint32_t zero = 0;
   if (cudaMemsetAsync(ctx->d_state, 0, 5 * (size_t)ctx->T * sizeof(uint32_t), st) != cudaSuccess ||
       cudaMemsetAsync(ctx->d_error, 0, sizeof(uint32_t), st) != cudaSuccess)
     return FP8ADAM_ERR_CUDA;
 #ifdef FP8ADAM_DEBUG
+  const uint32_t zero = 0;
   if (cudaMemcpyToSymbolAsync(g_debug_flags, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return FP8ADAM_ERR_CUDA;
 #endif
-  (void)zero;
   if (cudaStreamSynchronize(st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
   return bounds ? FP8ADAM_ERR_DEBUG_BOUNDS : FP8ADAM_ERR_DEVICE_TIMEOUT;
 }
