@@ -334,8 +334,8 @@ def our_arm(args):
                 "kernel_ms_max": max(kernel_ms),
                 "frac_of_8TBs_nominal": achieved / 8000.0}
 
-    cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
+    cpu = None  # the CPU oracle is timed on rank 0 of a 1-GPU run only
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
 
         oracle.build()
