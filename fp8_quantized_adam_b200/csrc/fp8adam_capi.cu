@@ -691,6 +691,7 @@ extern "C" int fp8adam_step_host(fp8adam_ctx* ctx, const fp8adam_step_params* pa
   const bool whole = needs_prepass(p);
   const int ng = whole ? 1 : G;
   NvtxRange range("fp8adam_step_host");
+  bool first = true;  // no chunk of this step has been launched yet (clears the JIT accumulators)
   for (int g = 0; g < ng; ++g) {
     const int32_t t0 = whole ? 0 : ctx->grp_tensor[(size_t)g];
     const int32_t t1 = whole ? ctx->T : ctx->grp_tensor[(size_t)g + 1];
@@ -705,8 +706,9 @@ extern "C" int fp8adam_step_host(fp8adam_ctx* ctx, const fp8adam_step_params* pa
       return FP8ADAM_ERR_CUDA;
     const int32_t c0 = whole ? 0 : ctx->grp_chunk[(size_t)g];
     const int32_t c1 = whole ? ctx->total_units : ctx->grp_chunk[(size_t)g + 1];
-    const int rc = run_step_range(ctx, p, st, c0, c1, g == 0);
+    const int rc = run_step_range(ctx, p, st, c0, c1, first);
     if (rc != FP8ADAM_OK) return rc;
+    if (c1 > c0) first = false;
   }
   if (amax_host && ctx->T > 0) {
     const size_t bytes = (size_t)ctx->T * sizeof(float);

@@ -290,13 +290,19 @@ def test_llama2_7b_layout_subset_3_steps():
         r.check_invariants()
 
 
+HOST_LAYOUTS = {"ragged": [70001, 0, 4096, 33, 3 * 65536 + 4099, 17, 200003, 1, 131072, 65535, 9000, 4097],
+                "empty_first": [0, 0, 0, 5000, 0, 17, 300000, 0]}
+
+
+@pytest.mark.parametrize("layout", list(HOST_LAYOUTS))
 @pytest.mark.parametrize("jit", [False, True], ids=["delayed", "jit_every_step"])
-def test_step_from_host_buffers(jit):
+def test_step_from_host_buffers(jit, layout):
     """fp8adam_step_host: gradients copied from pinned host memory by the
     library (the device buffer is zeroed before each step), the step of each
     tensor group overlapping the copies of the next groups; every element
-    against the oracle, and the amax read back to the host."""
-    sizes = [70001, 0, 4096, 33, 3 * 65536 + 4099, 17, 200003, 1, 131072, 65535, 9000, 4097]
+    against the oracle, and the amax read back to the host.  With empty
+    tensors first, the first group that launches clears the JIT amax."""
+    sizes = HOST_LAYOUTS[layout]
     specs = workloads.custom_layout(sizes)
     r = Run(specs, 14, host=True, jit_every_step=jit)
     for _ in range(4):
