@@ -7,6 +7,8 @@ only concrete optimizer call), torch's float8 casts, and brute force.
 import math
 
 import numpy as np
+from hypothesis import given, settings
+from hypothesis import strategies as st
 import pytest
 import torch
 
@@ -316,3 +318,29 @@ def test_nan_gradient_propagates_to_amax(orc):
     assert st.m[5] & 0x7F == 0x7F
     _step(st, _grad(n, 62), 3)  # a NaN amax keeps the previous scale
     assert float(st.scale_m[0]) == s_before
+
+
+@settings(max_examples=30, deadline=None)
+@given(lr=st.floats(1e-5, 1e-2), beta1=st.floats(0.0, 0.999), beta2=st.floats(0.5, 0.9999),
+       eps=st.floats(1e-10, 1e-4), wd=st.floats(0.0, 0.3), steps=st.integers(1, 6), seed=st.integers(0, 2**31))
+def test_fp32_moments_match_torch_adamw_any_hyperparameters(lr, beta1, beta2, eps, wd, steps, seed):
+    """The fp32-moment step against torch.optim.AdamW for random
+    hyper-parameters (a wrong bias correction, decay order or eps placement
+    shows up for some beta/eps/wd), teacher-forced from the oracle's state at
+    every step: params within 1e-6 of the update scale."""
+    import oracle as orc
+
+    hp = dict(lr=lr, beta1=beta1, beta2=beta2, eps=eps, wd=wd)
+    n = 257
+    rng = np.random.default_rng(seed)
+    p0 = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    s = orc.TensorState(p0, FP32, FP32)
+    for t in range(1, steps + 1):
+        g = _grad(n, seed + t)
+        forced = pins.TorchFakeQuantAdamW(s.p, FP32, FP32, **hp)
+        forced.mq, forced.vq = torch.from_numpy(s.m.copy()), torch.from_numpy(s.v.copy())
+        forced.t = t - 1
+        p_before = s.p.copy()
+        _step(s, g, t, hp=hp)
+        forced.step(g)
+        assert pins.params_close(s.p, forced.p, lr, 1, p_before=p_before)
