@@ -71,10 +71,30 @@ class FP8AdamW:
         self.m = moments(m, self.m_fmt)
         self.v = moments(v, self.v_fmt)
         T = len(self.params)
-        self.scale_m = scale_m if scale_m is not None else torch.ones(T, dtype=torch.float32, device=dev)
-        self.scale_v = scale_v if scale_v is not None else torch.ones(T, dtype=torch.float32, device=dev)
-        self.amax_m = amax_m if amax_m is not None else torch.zeros(T, dtype=torch.float32, device=dev)
-        self.amax_v = amax_v if amax_v is not None else torch.zeros(T, dtype=torch.float32, device=dev)
+
+        def check(bufs, dtype, what):
+            # the library reads and writes these through raw pointers: size,
+            # dtype, device and layout must be exactly as declared
+            if len(bufs) != T:
+                raise ValueError("%s: one buffer per param expected" % what)
+            for b, p in zip(bufs, self.params):
+                if b.dtype != dtype or b.numel() != p.numel() or b.device != dev or not b.is_contiguous():
+                    raise ValueError("%s: contiguous %s of %d elements on %s expected" % (what, dtype, p.numel(), dev))
+
+        check(self.m, torch.float32 if self.m_fmt == capi.FP32 else torch.uint8, "m")
+        check(self.v, torch.float32 if self.v_fmt == capi.FP32 else torch.uint8, "v")
+
+        def per_tensor(t, fill, what):
+            if t is None:
+                return torch.full((T,), fill, dtype=torch.float32, device=dev)
+            if t.dtype != torch.float32 or t.numel() != T or t.device != dev or not t.is_contiguous():
+                raise ValueError("%s: contiguous float32 [%d] on %s expected" % (what, T, dev))
+            return t
+
+        self.scale_m = per_tensor(scale_m, 1.0, "scale_m")
+        self.scale_v = per_tensor(scale_v, 1.0, "scale_v")
+        self.amax_m = per_tensor(amax_m, 0.0, "amax_m")
+        self.amax_v = per_tensor(amax_v, 0.0, "amax_v")
         self.lr, self.betas, self.eps, self.weight_decay = lr, tuple(betas), eps, weight_decay
         self.t = 0
         arr = (capi.fp8adam_tensor * T)()
@@ -92,8 +112,7 @@ class FP8AdamW:
         self.param_bf16 = list(param_bf16) if param_bf16 is not None else None
         bf16_arr = None
         if self.param_bf16 is not None:
-            if len(self.param_bf16) != T:
-                raise ValueError("need one bf16 output per param")
+            check(self.param_bf16, torch.bfloat16, "param_bf16")
             bf16_arr = (ctypes.c_void_p * T)(*[b.data_ptr() for b in self.param_bf16])
         opts = capi.fp8adam_options(self.scale_m.data_ptr(), self.scale_v.data_ptr(), self.amax_m.data_ptr(),
                                     self.amax_v.data_ptr(), self.m_fmt, self.v_fmt, flags, margin_m, margin_v,

@@ -311,3 +311,24 @@ def test_step_from_host_buffers(jit, layout):
         M = r.model
         assert torch.equal(r.amax_host[:len(specs)], M.amax_m.cpu()) and \
             torch.equal(r.amax_host[len(specs):], M.amax_v.cpu())
+
+
+def test_binding_rejects_mismatched_buffers():
+    """The torch binding checks every buffer it hands to the library: moment
+    dtype and size, per-tensor arrays, bf16 outputs."""
+    dev = torch.device("cuda:0")
+    p = [torch.zeros(100, device=dev)]
+    g = [torch.zeros(100, device=dev, dtype=torch.bfloat16)]
+    with pytest.raises(ValueError):
+        FP8AdamW(p, g, m=[torch.zeros(100, device=dev)])                        # fp32 m for E4M3
+    with pytest.raises(ValueError):
+        FP8AdamW(p, g, v=[torch.zeros(99, device=dev, dtype=torch.uint8)])     # wrong size
+    with pytest.raises(ValueError):
+        FP8AdamW(p, g, scale_m=torch.ones(2, device=dev))                      # T = 1
+    with pytest.raises(ValueError):
+        FP8AdamW(p, g, param_bf16=[torch.zeros(100, device=dev)])              # not bf16
+    with pytest.raises(ValueError):
+        FP8AdamW(p, g, m=[torch.zeros(200, device=dev, dtype=torch.uint8)[::2]])  # not contiguous
+    opt = FP8AdamW(p, g, m_fmt="fp32", m=[torch.zeros(100, device=dev)])       # fp32 m in fp32 mode
+    opt.step()
+    opt.close()
