@@ -493,9 +493,32 @@ fp8adam_gradnorm_partial_kernel(const StepArgs a, double* partial, unsigned long
   const TensorDesc td = a.tensors[ch.tensor];
   const int64_t e0 = ch.start, e1 = ch.start + ch.len;
   FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
-  int64_t scalar_from = e0;
-  if (td.aligned) {
-    for (int64_t i = e0 + (int64_t)threadIdx.x * kVec; i + kVec <= e1; i += kTile) {
+  const int64_t vec_end = td.aligned ? e0 + (e1 - e0) / kVec * kVec : e0;
+  // Fast path: each gradient widened to double (exact) and squared into the
+  // sum by one fused multiply-add (exact square, one rounding), with no
+  // per-element tests.  Zero adds nothing and a subnormal its exact square,
+  // as in sumsq1, and the order is the same, so the sum is the same.  An inf
+  // or NaN makes the sum non-finite: the thread then redoes its elements with
+  // sumsq1, which counts them instead.
+  for (int64_t i = e0 + (int64_t)threadIdx.x * kVec; i < vec_end; i += kTile) {
+    const uint4 g0 = ld_ro_u4(td.g + i);
+    const uint4 g1 = ld_ro_u4(td.g + i + 8);
+    const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const double lo = (double)bf16_lo(gw[k]);
+      const double hi = (double)bf16_hi(gw[k]);
+      acc = __fma_rn(lo, lo, acc);
+      acc = __fma_rn(hi, hi, acc);
+    }
+  }
+  for (int64_t i = vec_end + threadIdx.x; i < e1; i += kThreads) {
+    const double x = (double)__uint_as_float((uint32_t)td.g[i] << 16);
+    acc = __fma_rn(x, x, acc);
+  }
+  if (!isfinite(acc)) {  // a non-finite gradient in this thread's elements
+    acc = 0.0;
+    for (int64_t i = e0 + (int64_t)threadIdx.x * kVec; i < vec_end; i += kTile) {
       const uint4 g0 = ld_ro_u4(td.g + i);
       const uint4 g1 = ld_ro_u4(td.g + i + 8);
       const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
@@ -505,9 +528,8 @@ fp8adam_gradnorm_partial_kernel(const StepArgs a, double* partial, unsigned long
         sumsq1(gw[k] >> 16, acc, bad);
       }
     }
-    scalar_from = e0 + (e1 - e0) / kVec * kVec;
+    for (int64_t i = vec_end + threadIdx.x; i < e1; i += kThreads) sumsq1(td.g[i], acc, bad);
   }
-  for (int64_t i = scalar_from + threadIdx.x; i < e1; i += kThreads) sumsq1(td.g[i], acc, bad);
   const double s = block_sum_d(acc, red);
   const uint32_t nb = block_sum(bad, redi);
   if (threadIdx.x == 0) {
