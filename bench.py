@@ -333,6 +333,9 @@ def our_arm(args):
                 "kernel_ms_p90": sorted(kernel_ms)[min(len(kernel_ms) - 1, (9 * len(kernel_ms)) // 10)],
                 "kernel_ms_max": max(kernel_ms),
                 "frac_of_8TBs_nominal": achieved / 8000.0}
+    if args.variant == "sr":
+        roofline["note"] = ("stochastic rounding is bound by instruction issue, not DRAM (Philox4x32-10 and the exact "
+                            "SR encoder): profiles/fp8adam_step_ext_tma_kernel_sr_llama2_100m.md")
 
     cpu = None  # the CPU oracle is timed on rank 0 of a 1-GPU run only
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
