@@ -40,8 +40,8 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum per element of the step kernel,
 # from the ncu capture summarised in profiles/, valid while the kernel sources
 # hash to KERNEL_SHA (null otherwise).
-TRAFFIC_PER_PARAM = 13.4743  # profiles/fp8adam_step_tma_kernel_llama2_100m.md: 876.40 MB + 599.43 MB / 109.53 M
-KERNEL_SHA = "4e8f94d3fc05ec54"
+TRAFFIC_PER_PARAM = 13.4859  # profiles/fp8adam_step_tma_kernel_llama2_100m.md: 876.40 MB + 600.71 MB / 109.53 M
+KERNEL_SHA = "e2bd44da06c55c97"
 
 
 def kernel_sha() -> str:

@@ -23,6 +23,7 @@ ERR_NOALLOC_LIMIT = -6
 ERR_DEVICE_TIMEOUT = -7
 ERR_DEBUG_BOUNDS = -8
 ERR_OVERLAP = -9
+ERR_SCHEDULE_END = -10
 NOALLOC_MAX_TENSORS = 4096
 
 E4M3, E5M2, FP32 = 0, 1, 2
@@ -125,6 +126,12 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.fp8adam_step_noalloc.restype = ctypes.c_int
     L.fp8adam_step_noalloc.argtypes = [ctypes.POINTER(fp8adam_tensor), i32, vp, vp, vp, vp, i32, i32, u32,
                                        f, f, f, f, f, i64, vp]
+    L.fp8adam_set_schedule.restype = ctypes.c_int
+    L.fp8adam_set_schedule.argtypes = [vp, ctypes.POINTER(fp8adam_step_params), i32, vp]
+    L.fp8adam_step_scheduled.restype = ctypes.c_int
+    L.fp8adam_step_scheduled.argtypes = [vp, vp]
+    L.fp8adam_get_schedule_step.restype = ctypes.c_int
+    L.fp8adam_get_schedule_step.argtypes = [vp, ctypes.POINTER(ctypes.c_int64), vp]
     L.fp8adam_debug_inject_wait.restype = ctypes.c_int
     L.fp8adam_debug_inject_wait.argtypes = [i32, i32]
     L.fp8adam_debug_set_numel.restype = ctypes.c_int
@@ -207,6 +214,22 @@ def fp8adam_step_host(ctx, params: fp8adam_step_params, host_grads, amax_host: i
                                                         cuda_stream))
 
 
+def fp8adam_set_schedule(ctx, steps, cuda_stream: int) -> None:
+    """steps: a sequence of fp8adam_step_params for consecutive steps."""
+    arr = (fp8adam_step_params * len(steps))(*steps)
+    _check("fp8adam_set_schedule", lib().fp8adam_set_schedule(ctx, arr, len(steps), cuda_stream))
+
+
+def fp8adam_step_scheduled(ctx, cuda_stream: int) -> None:
+    _check("fp8adam_step_scheduled", lib().fp8adam_step_scheduled(ctx, cuda_stream))
+
+
+def fp8adam_get_schedule_step(ctx, cuda_stream: int) -> int:
+    t = ctypes.c_int64(0)
+    _check("fp8adam_get_schedule_step", lib().fp8adam_get_schedule_step(ctx, ctypes.byref(t), cuda_stream))
+    return int(t.value)
+
+
 def fp8adam_encode_sr(fmt: int, x: int, r: int, out: int, n: int, cuda_stream: int) -> None:
     _check("fp8adam_encode_sr", lib().fp8adam_encode_sr(fmt, x, r, out, n, cuda_stream))
 
@@ -233,4 +256,5 @@ EXPORTED = ["fp8adam_create", "fp8adam_step", "fp8adam_get_stats", "fp8adam_rese
             "fp8adam_destroy", "fp8adam_strerror", "fp8adam_encode", "fp8adam_encode_bits_range",
             "fp8adam_decode", "fp8adam_launch_count", "fp8adam_step_noalloc", "fp8adam_create_ex",
             "fp8adam_step_ex", "fp8adam_get_grad_info", "fp8adam_check", "fp8adam_encode_sr", "fp8adam_step_host",
-            "fp8adam_debug_inject_wait", "fp8adam_debug_set_numel"]
+            "fp8adam_debug_inject_wait", "fp8adam_debug_set_numel", "fp8adam_set_schedule",
+            "fp8adam_step_scheduled", "fp8adam_get_schedule_step"]

@@ -186,6 +186,39 @@ ExtFn pick_amax_ext(int mf, int vf) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Constants of step t: computed in double, rounded once to fp32.
+StepConsts make_consts(const fp8adam_step_params& p) {
+  const double bc1 = 1.0 - std::pow((double)p.beta1, (double)p.step);
+  const double bc2 = 1.0 - std::pow((double)p.beta2, (double)p.step);
+  StepConsts c;
+  c.b1 = p.beta1;
+  c.omb1 = (float)(1.0 - (double)p.beta1);
+  c.b2 = p.beta2;
+  c.omb2 = (float)(1.0 - (double)p.beta2);
+  c.step_size = (float)((double)p.lr / bc1);
+  c.isbc2 = (float)(1.0 / std::sqrt(bc2));
+  c.eps = p.eps;
+  c.decay = (float)(1.0 - (double)p.lr * (double)p.weight_decay);
+  return c;
+}
+
+// A scheduled step's first kernel (one thread): copy the entry of the
+// device step counter to `cur` and advance the counter; past the end of the
+// schedule, mark `cur` invalid (the step's kernels then do nothing) and set
+// bit 1 of the error word.
+__global__ void sched_select_kernel(const SchedEntry* sched, int64_t first, int32_t count, int64_t* next_step,
+                                    SchedEntry* cur, uint32_t* err) {
+  const int64_t k = *next_step - first;
+  if (k < 0 || k >= count) {
+    cur->valid = 0;
+    atomicOr(err, 2u);
+    return;
+  }
+  *cur = sched[k];
+  cur->valid = 1;
+  *next_step += 1;
+}
+
 // True if two of the byte ranges overlap and at least one of them is
 // written.  Sorted by start, a range overlaps an earlier one iff it starts
 // before the furthest end seen so far (of any range if it is written, of
@@ -251,6 +284,15 @@ struct fp8adam_ctx {
   std::vector<int32_t> grp_tensor;    // [G+1] first tensor of each group
   std::vector<int32_t> grp_chunk;     // [G+1] first chunk of each group
   cudaStream_t copy_stream = nullptr; // created on first use
+  // fp8adam_set_schedule / fp8adam_step_scheduled: the entries of steps
+  // sched_first .. sched_first + sched_count - 1, the device step counter and
+  // the entry of the step in flight
+  SchedEntry* d_sched = nullptr;
+  int32_t sched_cap = 0, sched_count = 0;
+  int64_t sched_first = 0;
+  bool sched_prepass = false;         // some entry needs the grad-norm pre-pass
+  int64_t* d_next_step = nullptr;
+  SchedEntry* d_cur = nullptr;
   cudaEvent_t start_event = nullptr;
   std::vector<cudaEvent_t> grp_event; // [G] the group's copies are done
 };
@@ -268,6 +310,9 @@ static void free_ctx(fp8adam_ctx* c) {
   cudaFree(c->d_norm);
   cudaFree(c->d_state);
   cudaFree(c->d_stats);
+  cudaFree(c->d_sched);
+  cudaFree(c->d_next_step);
+  cudaFree(c->d_cur);
   for (cudaEvent_t e : c->grp_event)
     if (e) cudaEventDestroy(e);
   if (c->start_event) cudaEventDestroy(c->start_event);
@@ -500,24 +545,18 @@ static bool needs_prepass(const fp8adam_step_params& p) {
 // `first`: the range is the step's first, so the JIT accumulators are
 // cleared before it.  The grad-norm pre-pass needs all gradients: with it
 // the range is the whole table.
+// `cur` (a scheduled step): the kernels take the constants and per-step
+// options from that device entry instead of `p`; whether the pre-passes run
+// is then decided per schedule (grad norm) or per context (JIT amax).
 static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t st, int32_t c0, int32_t c1,
-                          bool first) {
+                          bool first, const SchedEntry* cur = nullptr) {
   if (c1 <= c0) return FP8ADAM_OK;  // only empty tensors
-  const bool prepass = needs_prepass(p);
+  const bool prepass = cur ? ctx->sched_prepass : needs_prepass(p);
   const bool ext = ctx->ext || prepass;
 
-  // constants of step t: double, rounded once to fp32
-  const double bc1 = 1.0 - std::pow((double)p.beta1, (double)p.step);
-  const double bc2 = 1.0 - std::pow((double)p.beta2, (double)p.step);
   StepArgs a;
-  a.c.b1 = p.beta1;
-  a.c.omb1 = (float)(1.0 - (double)p.beta1);
-  a.c.b2 = p.beta2;
-  a.c.omb2 = (float)(1.0 - (double)p.beta2);
-  a.c.step_size = (float)((double)p.lr / bc1);
-  a.c.isbc2 = (float)(1.0 / std::sqrt(bc2));
-  a.c.eps = p.eps;
-  a.c.decay = (float)(1.0 - (double)p.lr * (double)p.weight_decay);
+  a.c = make_consts(p);
+  a.cur = cur;
 
   const size_t T = (size_t)ctx->T;
   uint32_t* acc_m = ctx->d_state;
@@ -537,7 +576,7 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
   a.acc_v = acc_v;
 
   const dim3 block(kThreads), grid((unsigned)(c1 - c0));
-  const bool jit = p.step == 1 || (ctx->flags & FP8ADAM_FLAG_JIT_EVERY_STEP);
+  const bool jit = (!cur && p.step == 1) || (ctx->flags & FP8ADAM_FLAG_JIT_EVERY_STEP);
   const bool stats = (ctx->flags & FP8ADAM_FLAG_STATS) != 0;
   if (!ext) {
     if (jit) {
@@ -586,7 +625,7 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
       return FP8ADAM_ERR_CUDA;
     fp8adam_gradnorm_partial_kernel<<<grid, block, 0, st>>>(a, ctx->d_partial, ctx->d_nonfinite);
     fp8adam_gradnorm_finalize_kernel<<<1, block, 0, st>>>(ctx->d_partial, (int)(c1 - c0), ctx->d_nonfinite,
-                                                          p.loss_scale, p.max_norm, p.skip_nonfinite,
+                                                          p.loss_scale, p.max_norm, p.skip_nonfinite, cur,
                                                           ctx->d_grad_mult, ctx->d_skip, ctx->d_norm);
     g_launches.fetch_add(2, std::memory_order_relaxed);
     e.grad_mult = ctx->d_grad_mult;
@@ -651,6 +690,99 @@ extern "C" int fp8adam_step_ex(fp8adam_ctx* ctx, const fp8adam_step_params* para
       std::isinf(p.max_norm))
     return FP8ADAM_ERR_INVALID_ARG;
   return run_step(ctx, p, static_cast<cudaStream_t>(cuda_stream));
+}
+
+static bool valid_step_params(const fp8adam_step_params& p) {
+  return valid_hparams(p.lr, p.beta1, p.beta2, p.eps, p.weight_decay, p.step) && p.loss_scale > 0.0f &&
+         std::isfinite(p.loss_scale) && !std::isnan(p.max_norm) && !std::isinf(p.max_norm);
+}
+
+extern "C" int fp8adam_set_schedule(fp8adam_ctx* ctx, const fp8adam_step_params* steps, int32_t count,
+                                    void* cuda_stream) {
+  if (!ctx || !steps || count < 1) return FP8ADAM_ERR_INVALID_ARG;
+  const int64_t first = steps[0].step;
+  // step 1 takes the amax pre-pass decided on the host, so a schedule starts
+  // after it unless every step has the pre-pass (current scaling)
+  if (first < 2 && !(ctx->flags & FP8ADAM_FLAG_JIT_EVERY_STEP)) return FP8ADAM_ERR_INVALID_ARG;
+  std::vector<SchedEntry> host;
+  try {
+    host.resize((size_t)count);
+  } catch (...) {
+    return FP8ADAM_ERR_OOM;
+  }
+  bool prepass = false;
+  for (int32_t k = 0; k < count; ++k) {
+    const fp8adam_step_params& p = steps[k];
+    if (!valid_step_params(p) || p.step != first + k) return FP8ADAM_ERR_INVALID_ARG;
+    SchedEntry& e = host[(size_t)k];
+    e.c = make_consts(p);
+    e.loss_scale = p.loss_scale;
+    e.max_norm = p.max_norm;
+    e.skip_nonfinite = p.skip_nonfinite ? 1 : 0;
+    e.t_lo = (uint32_t)p.step;
+    e.hist_slot = ctx->hist_len ? (int32_t)((p.step - 1) % ctx->hist_len) : 0;
+    e.valid = 1;
+    prepass = prepass || needs_prepass(p);
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP8ADAM_ERR_CUDA;
+  if (dev != ctx->device) return FP8ADAM_ERR_WRONG_DEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  // the steps already queued may still read the old schedule
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
+  if (count > ctx->sched_cap) {
+    cudaFree(ctx->d_sched);
+    ctx->d_sched = nullptr;
+    ctx->sched_cap = 0;
+    if (cudaMalloc(&ctx->d_sched, (size_t)count * sizeof(SchedEntry)) != cudaSuccess) {
+      cudaGetLastError();
+      return FP8ADAM_ERR_OOM;
+    }
+    ctx->sched_cap = count;
+  }
+  if ((!ctx->d_next_step && cudaMalloc(&ctx->d_next_step, sizeof(int64_t)) != cudaSuccess) ||
+      (!ctx->d_cur && cudaMalloc(&ctx->d_cur, sizeof(SchedEntry)) != cudaSuccess)) {
+    cudaGetLastError();
+    return FP8ADAM_ERR_OOM;
+  }
+  if (cudaMemcpy(ctx->d_sched, host.data(), (size_t)count * sizeof(SchedEntry), cudaMemcpyHostToDevice) !=
+          cudaSuccess ||
+      cudaMemcpy(ctx->d_next_step, &first, sizeof(first), cudaMemcpyHostToDevice) != cudaSuccess)
+    return FP8ADAM_ERR_CUDA;
+  ctx->sched_first = first;
+  ctx->sched_count = count;
+  ctx->sched_prepass = prepass;
+  return FP8ADAM_OK;
+}
+
+extern "C" int fp8adam_step_scheduled(fp8adam_ctx* ctx, void* cuda_stream) {
+  if (!ctx || ctx->sched_count == 0) return FP8ADAM_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP8ADAM_ERR_CUDA;
+  if (dev != ctx->device) return FP8ADAM_ERR_WRONG_DEVICE;
+  if (ctx->total_units == 0) return FP8ADAM_OK;
+  NvtxRange range("fp8adam_step_scheduled");
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  sched_select_kernel<<<1, 1, 0, st>>>(ctx->d_sched, ctx->sched_first, ctx->sched_count, ctx->d_next_step,
+                                       ctx->d_cur, ctx->d_error);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  // the host-side parameters only fill the unused kernel arguments
+  fp8adam_step_params p;
+  std::memset(&p, 0, sizeof(p));
+  p.lr = 0.0f;
+  p.beta1 = p.beta2 = 0.5f;
+  p.step = 2;
+  p.loss_scale = 1.0f;
+  return run_step_range(ctx, p, st, 0, ctx->total_units, true, ctx->d_cur);
+}
+
+extern "C" int fp8adam_get_schedule_step(fp8adam_ctx* ctx, int64_t* next_step, void* cuda_stream) {
+  if (!ctx || !next_step || !ctx->d_next_step) return FP8ADAM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaMemcpyAsync(next_step, ctx->d_next_step, sizeof(int64_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return FP8ADAM_ERR_CUDA;
+  return FP8ADAM_OK;
 }
 
 extern "C" int fp8adam_step_host(fp8adam_ctx* ctx, const fp8adam_step_params* params,
@@ -777,7 +909,8 @@ extern "C" int fp8adam_check(fp8adam_ctx* ctx, void* cuda_stream) {
     return FP8ADAM_ERR_CUDA;
 #endif
   if (cudaStreamSynchronize(st) != cudaSuccess) return FP8ADAM_ERR_CUDA;
-  return bounds ? FP8ADAM_ERR_DEBUG_BOUNDS : FP8ADAM_ERR_DEVICE_TIMEOUT;
+  if (bounds) return FP8ADAM_ERR_DEBUG_BOUNDS;
+  return (e & 1u) ? FP8ADAM_ERR_DEVICE_TIMEOUT : FP8ADAM_ERR_SCHEDULE_END;
 }
 
 extern "C" int fp8adam_debug_inject_wait(int32_t cta, int32_t subtile) {
@@ -824,6 +957,7 @@ extern "C" const char* fp8adam_strerror(int code) {
     case FP8ADAM_ERR_CUDA: return "CUDA runtime error";
     case FP8ADAM_ERR_DEBUG_BOUNDS: return "a kernel access outside its tensor was skipped (debug build)";
     case FP8ADAM_ERR_OVERLAP: return "a written buffer (param, m, v or bf16 copy) overlaps another buffer";
+    case FP8ADAM_ERR_SCHEDULE_END: return "a scheduled step ran past the end of its schedule (nothing was updated)";
     case FP8ADAM_ERR_OOM: return "device allocation failed";
     case FP8ADAM_ERR_WRONG_DEVICE: return "current device differs from the context's";
     case FP8ADAM_ERR_NOALLOC_LIMIT: return "more tensors than the allocation-free step holds (FP8ADAM_NOALLOC_MAX_TENSORS)";

@@ -58,8 +58,8 @@ __device__ __forceinline__ uint4 philox_round(uint4 c, uint32_t k0, uint32_t k1)
 
 // random words of elements (2q, 2q+1) of tensor ti at this step:
 // .x/.y -> element 2q (m, v); .z/.w -> element 2q+1 (m, v)
-__device__ __forceinline__ uint4 sr_words(const ExtArgs& a, int ti, int64_t q) {
-  uint4 c = make_uint4((uint32_t)q, (uint32_t)((uint64_t)q >> 32), (uint32_t)ti, a.t_lo);
+__device__ __forceinline__ uint4 sr_words(const ExtArgs& a, int ti, uint32_t t_lo, int64_t q) {
+  uint4 c = make_uint4((uint32_t)q, (uint32_t)((uint64_t)q >> 32), (uint32_t)ti, t_lo);
 #pragma unroll
   for (int r = 0; r < 10; ++r) c = philox_round(c, a.sr_key[r][0], a.sr_key[r][1]);
   return c;
@@ -72,12 +72,12 @@ __device__ __forceinline__ uint4 sr_words(const ExtArgs& a, int ti, int64_t q) {
 struct SrChunk {
   uint32_t x1, y1, w1;
 };
-__device__ __forceinline__ SrChunk sr_chunk(const ExtArgs& a, int ti, int64_t q0) {
+__device__ __forceinline__ SrChunk sr_chunk(const ExtArgs& a, int ti, uint32_t t_lo, int64_t q0) {
   const uint64_t p1 = (uint64_t)kPhiloxM1 * (uint32_t)ti;
   SrChunk u;
   u.x1 = (uint32_t)(p1 >> 32) ^ (uint32_t)((uint64_t)q0 >> 32) ^ a.sr_key[0][0];
   u.y1 = (uint32_t)p1;
-  u.w1 = a.t_lo ^ a.sr_key[0][1];
+  u.w1 = t_lo ^ a.sr_key[0][1];
   return u;
 }
 __device__ __forceinline__ uint4 sr_words_chunk(const ExtArgs& a, const SrChunk& u, uint32_t q_lo) {
@@ -173,9 +173,12 @@ __device__ __forceinline__ float ext_q(const ExtArgs& a, float x, float s, float
 }
 
 struct ExtSeg {  // per tensor segment
+  StepConsts c;   // the step's constants (argument or schedule entry)
   float inv_s_m, inv_s_v, s_m_new, s_v_new, inv_s_m_new, inv_s_v_new, gm;
   uint16_t* pb;
   int ti;
+  uint32_t t_lo;      // the step, for the SR counter
+  int32_t hist_slot;  // this step's slot of the amax history ring
 };
 
 // One element (tails, unaligned tensors).
@@ -183,10 +186,10 @@ template <int MF, int VF, bool STATS, int SRM>
 __device__ __forceinline__ void ext_element(const ExtArgs& a, const TensorDesc& td, const ExtSeg& sg, int64_t i,
                                             float& am, float& av, uint32_t& flushed, uint32_t& sat) {
   FP8ADAM_BOUNDS(i >= 0 && i < td.numel);
-  const StepConsts& c = a.s.c;
+  const StepConsts& c = sg.c;
   uint32_t rm = 0, rv = 0;
   if (use_sr<SRM>(a)) {
-    const uint4 r = sr_words(a, sg.ti, i >> 1);
+    const uint4 r = sr_words(a, sg.ti, sg.t_lo, i >> 1);
     rm = (i & 1) ? r.z : r.x;
     rv = (i & 1) ? r.w : r.y;
   }
@@ -210,7 +213,7 @@ template <int MF, int VF, bool STATS, int SRM>
 __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& td, const ExtSeg& sg, int64_t i,
                                             float& am, float& av, uint32_t& flushed, uint32_t& sat) {
   FP8ADAM_BOUNDS(i >= 0 && i + kVec <= td.numel);
-  const StepConsts& c = a.s.c;
+  const StepConsts& c = sg.c;
   float4 pv[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) pv[k] = ld_stream_f4(td.p + i + 4 * k);
@@ -231,8 +234,8 @@ __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& 
                         __fmul_rn(bf16_lo(gw[2 * k + 1]), sg.gm), __fmul_rn(bf16_hi(gw[2 * k + 1]), sg.gm)};
     uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
     if (use_sr<SRM>(a)) {
-      r0 = sr_words(a, sg.ti, (i + 4 * k) >> 1);
-      r1 = sr_words(a, sg.ti, ((i + 4 * k) >> 1) + 1);
+      r0 = sr_words(a, sg.ti, sg.t_lo, (i + 4 * k) >> 1);
+      r1 = sr_words(a, sg.ti, sg.t_lo, ((i + 4 * k) >> 1) + 1);
     }
     const uint32_t rmj[4] = {r0.x, r0.z, r1.x, r1.z};
     const uint32_t rvj[4] = {r0.y, r0.w, r1.y, r1.w};
@@ -278,6 +281,15 @@ __device__ __forceinline__ ExtSeg ext_setup(const ExtArgs& a, int ti, float gm) 
   ExtSeg sg;
   sg.ti = ti;
   sg.gm = gm;
+  if (S.cur != nullptr) {  // a scheduled step (the kernel checked that the entry is valid)
+    sg.c = S.cur->c;
+    sg.t_lo = S.cur->t_lo;
+    sg.hist_slot = S.cur->hist_slot;
+  } else {
+    sg.c = S.c;
+    sg.t_lo = a.t_lo;
+    sg.hist_slot = a.hist_slot;
+  }
   sg.pb = a.p_bf16 ? a.p_bf16[ti] : nullptr;
   const float s_m = S.scale_m[ti], s_v = S.scale_v[ti];
   float am_in = __uint_as_float(S.amax_in_m[ti]);
@@ -351,8 +363,8 @@ __device__ __forceinline__ void ext_flush(const ExtArgs& a, int ti, int32_t nuni
       S.amax_m[ti] = __uint_as_float(fm);
       S.amax_v[ti] = __uint_as_float(fv);
       if (a.hist_m) {
-        a.hist_m[(int64_t)a.hist_slot * S.num_tensors + ti] = __uint_as_float(fm);
-        a.hist_v[(int64_t)a.hist_slot * S.num_tensors + ti] = __uint_as_float(fv);
+        a.hist_m[(int64_t)sg.hist_slot * S.num_tensors + ti] = __uint_as_float(fm);
+        a.hist_v[(int64_t)sg.hist_slot * S.num_tensors + ti] = __uint_as_float(fv);
       }
       S.scale_m[ti] = sg.s_m_new;
       S.scale_v[ti] = sg.s_v_new;
@@ -368,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 fp8adam_step_ext_kernel(const ExtArgs a) {
   __shared__ uint32_t red[4][kThreads / 32];
   if (a.skip && *a.skip) return;  // a non-finite gradient: the step is skipped
+  if (a.s.cur && !a.s.cur->valid) return;  // the schedule ran out
   const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
   const Chunk ch = a.s.chunks[blockIdx.x];
   const int ti = ch.tensor;
@@ -391,6 +404,8 @@ fp8adam_amax_ext_kernel(const ExtArgs a) {
   __shared__ uint32_t red[2][kThreads / 32];
   if (a.skip && *a.skip) return;
   const StepArgs& S = a.s;
+  StepConsts c;
+  if (!step_consts(S, c)) return;
   const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
   const Chunk ch = S.chunks[blockIdx.x];
   const int ti = ch.tensor;
@@ -421,7 +436,7 @@ fp8adam_amax_ext_kernel(const ExtArgs a) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           float mn, vn;
-          moments(S.c, g[j], mo[j], vo[j], mn, vn);
+          moments(c, g[j], mo[j], vo[j], mn, vn);
           am = fmax_nan(am, fabsf(mn));
           av = fmax_nan(av, fabsf(vn));
         }
@@ -432,7 +447,7 @@ fp8adam_amax_ext_kernel(const ExtArgs a) {
   for (int64_t i = scalar_from + threadIdx.x; i < e1; i += kThreads) {
     const float g = __fmul_rn(__uint_as_float((uint32_t)td.g[i] << 16), gm);
     float mn, vn;
-    moments(S.c, g, load1<MF>(td.m, i, inv_s_m), load1<VF>(td.v, i, inv_s_v), mn, vn);
+    moments(c, g, load1<MF>(td.m, i, inv_s_m), load1<VF>(td.v, i, inv_s_v), mn, vn);
     am = fmax_nan(am, fabsf(mn));
     av = fmax_nan(av, fabsf(vn));
   }
@@ -538,19 +553,29 @@ fp8adam_gradnorm_partial_kernel(const StepArgs a, double* partial, unsigned long
   }
 }
 
-// One CTA: the fixed-order total, the multiplier and the skip flag.
+// One CTA: the fixed-order total, the multiplier and the skip flag (the
+// options from `cur` on a scheduled step).
 // c = (1/loss_scale) * min(1, max_norm / (norm + 1e-6)), norm = sqrt(sum)/loss_scale
 // (clip_grad_norm_'s definition on the unscaled gradients); max_norm <= 0 =
 // no clipping; all in double, c rounded once to fp32.
 __global__ void __launch_bounds__(kThreads)
 fp8adam_gradnorm_finalize_kernel(const double* partial, int n, const unsigned long long* nonfinite,
-                                 float loss_scale, float max_norm, int skip_nonfinite, float* grad_mult,
-                                 uint32_t* skip, double* norm_out) {
+                                 float loss_scale, float max_norm, int skip_nonfinite, const SchedEntry* cur,
+                                 float* grad_mult, uint32_t* skip, double* norm_out) {
   __shared__ double red[kThreads / 32];
   double acc = 0.0;
   for (int k = threadIdx.x; k < n; k += kThreads) acc = __dadd_rn(acc, partial[k]);
   const double sum = block_sum_d(acc, red);
   if (threadIdx.x == 0) {
+    if (cur != nullptr) {  // a scheduled step: the options of its entry
+      if (!cur->valid) {
+        *skip = 1u;  // the schedule ran out: nothing is updated
+        return;
+      }
+      loss_scale = cur->loss_scale;
+      max_norm = cur->max_norm;
+      skip_nonfinite = cur->skip_nonfinite;
+    }
     const double inv = __ddiv_rn(1.0, (double)loss_scale);
     const double norm = __dmul_rn(__dsqrt_rn(sum), inv);
     double coef = 1.0;

@@ -44,7 +44,7 @@ __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& s
                                              const ExtSeg& sg, const SrChunk& su, int64_t i, float& am, float& av,
                                              uint32_t& flushed, uint32_t& sat) {
   FP8ADAM_BOUNDS(i >= 0 && i + 4 <= td.numel);
-  const StepConsts& c = a.s.c;
+  const StepConsts& c = sg.c;
   const float4 pin = *reinterpret_cast<const float4*>(&st.p[j]);
   const uint2 gq = *reinterpret_cast<const uint2*>(&st.g[j]);
   const uint32_t mw = *reinterpret_cast<const uint32_t*>(&st.m[j]);
@@ -125,6 +125,7 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
 
   if (*(volatile const uint32_t*)err) return;  // an earlier CTA timed out: stop at once
   if (a.skip && *a.skip) return;              // a non-finite gradient: the step is skipped
+  if (a.s.cur && !a.s.cur->valid) return;     // the schedule ran out
   const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
   const Chunk ch = a.s.chunks[blockIdx.x];
   const int ti = ch.tensor;
@@ -137,7 +138,7 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   uint32_t flushed = 0, sat = 0;
 
   SrChunk su{0u, 0u, 0u};
-  if constexpr (SR) su = sr_chunk(a, ti, e0 >> 1);
+  if constexpr (SR) su = sr_chunk(a, ti, sg.t_lo, e0 >> 1);
   const int nsub = ext_vec_ok(td, sg) ? (int)((e1 - e0) / kSub) : 0;
   if (!tma_stream(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
         ext_consume4<MF, VF, STATS, SR>(a, st, j, td, sg, su, i, am, av, flushed, sat);

@@ -63,6 +63,19 @@ struct StepConsts {
   float b1, omb1, b2, omb2, step_size, isbc2, eps, decay;
 };
 
+// One step of a device-side schedule (fp8adam_set_schedule): the constants
+// and per-step options, computed on the host; the step reads the entry the
+// schedule's select kernel copied for it (valid = 0: the schedule ran out,
+// and the step does nothing).
+struct SchedEntry {
+  StepConsts c;
+  float loss_scale, max_norm;
+  int32_t skip_nonfinite;
+  uint32_t t_lo;      // the step (stochastic rounding's counter word)
+  int32_t hist_slot;  // (t - 1) % amax history length
+  int32_t valid;
+};
+
 struct StepArgs {
   const TensorDesc* tensors;     // [T]
   const Chunk* chunks;           // [chunks] tensor and start of each chunk (one per CTA)
@@ -78,7 +91,20 @@ struct StepArgs {
   uint32_t* done;            // [T] finished-tile counters, zero between steps
   unsigned long long* stats; // [2] flushed, saturated (STATS only)
   StepConsts c;
+  const SchedEntry* cur;     // scheduled step: constants from here; else null (use c)
 };
+
+// The step's constants: the kernel argument, or the current schedule entry.
+// False when the schedule has run out (the kernel then does nothing).
+__device__ __forceinline__ bool step_consts(const StepArgs& a, StepConsts& c) {
+  if (a.cur == nullptr) {
+    c = a.c;
+    return true;
+  }
+  if (!a.cur->valid) return false;
+  c = a.cur->c;
+  return true;
+}
 
 // ------------------------------------------------------------ memory access
 __device__ __forceinline__ float4 ld_stream_f4(const float* p) {
@@ -328,7 +354,8 @@ __device__ __forceinline__ void run_segment(const StepArgs& a, int ti, int64_t e
   FP8ADAM_BOUNDS(ti >= 0 && ti < a.num_tensors);
   const TensorDesc td = a.tensors[ti];
   FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
-  const StepConsts c = a.c;
+  StepConsts c;
+  if (!step_consts(a, c)) return;
   const float s_m = a.scale_m[ti];
   const float s_v = a.scale_v[ti];
   float s_m_new = s_m, s_v_new = s_v;

@@ -206,7 +206,8 @@ fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
   const int ti = ch.tensor;
   FP8ADAM_BOUNDS(ti >= 0 && ti < a.num_tensors);
   const TensorDesc td = a.tensors[ti];
-  const StepConsts c = a.c;
+  StepConsts c;
+  if (!step_consts(a, c)) return;
   const int64_t e0 = ch.start, e1 = ch.start + ch.len;
   FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
   const float s_m = a.scale_m[ti];

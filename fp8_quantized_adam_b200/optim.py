@@ -177,6 +177,33 @@ class FP8AdamW:
             self.t -= 1
             raise
 
+    def set_schedule(self, lrs: Sequence[float], first_step: Optional[int] = None, loss_scale: float = 1.0,
+                     max_norm: float = 0.0, skip_nonfinite: bool = False,
+                     stream: Optional[torch.cuda.Stream] = None) -> None:
+        """Upload the parameters of steps first_step .. first_step + len(lrs)
+        - 1 (default: the step after the last one run) with learning rate
+        lrs[k] for step first_step + k, for ``step_scheduled``."""
+        first = self.t + 1 if first_step is None else int(first_step)
+        steps = [capi.fp8adam_step_params(float(lr), self.betas[0], self.betas[1], self.eps, self.weight_decay,
+                                          first + k, loss_scale, max_norm, 1 if skip_nonfinite else 0)
+                 for k, lr in enumerate(lrs)]
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        capi.fp8adam_set_schedule(self.ctx, steps, s.cuda_stream)
+
+    def step_scheduled(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """The next step of the schedule, with no per-step host state: can be
+        captured in a CUDA graph (torch.cuda.graph) and replayed.  ``self.t``
+        does not follow graph replays; ``scheduled_step()`` reads the device
+        counter."""
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        capi.fp8adam_step_scheduled(self.ctx, s.cuda_stream)
+        self.t += 1
+
+    def scheduled_step(self, stream: Optional[torch.cuda.Stream] = None) -> int:
+        """The step the next scheduled step will run (synchronises the stream)."""
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        return capi.fp8adam_get_schedule_step(self.ctx, s.cuda_stream)
+
     def grad_info(self, stream: Optional[torch.cuda.Stream] = None):
         """(global grad L2 norm, skipped) of the last step with a gradient
         pre-pass (synchronises the stream)."""

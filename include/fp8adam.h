@@ -69,6 +69,7 @@ extern "C" {
 #define FP8ADAM_ERR_DEVICE_TIMEOUT (-7)  /* a kernel's bounded wait ran out (see fp8adam_check) */
 #define FP8ADAM_ERR_DEBUG_BOUNDS (-8)    /* debug build: an access outside its tensor was skipped */
 #define FP8ADAM_ERR_OVERLAP (-9)         /* create: a written buffer overlaps another buffer */
+#define FP8ADAM_ERR_SCHEDULE_END (-10)   /* a scheduled step ran past its schedule (see fp8adam_check) */
 
 /* Storage format of a moment. */
 typedef enum {
@@ -258,6 +259,42 @@ int fp8adam_step_ex(fp8adam_ctx* ctx, const fp8adam_step_params* params,
 int fp8adam_step_host(fp8adam_ctx* ctx, const fp8adam_step_params* params,
                       const uint16_t* const* host_grads, float* amax_host,
                       void* cuda_stream);
+
+/* ---- steps that can be captured in a CUDA graph ------------------------
+ * fp8adam_step and fp8adam_step_ex pass the step's constants (t, lr, ...) as
+ * kernel arguments, so a captured launch would replay the same step.  A
+ * scheduled step instead takes them from device memory:
+ *
+ * fp8adam_set_schedule: steps[k] (host array, count >= 1) are the parameters
+ * of steps first .. first + count - 1 (steps[k].step = steps[0].step + k,
+ * each valid as for fp8adam_step_ex; lr and the other values may change from
+ * step to step, e.g. a learning-rate schedule).  Their constants are computed
+ * on the host exactly as fp8adam_step_ex computes them and copied to the
+ * device, and the context's device step counter is set to steps[0].step.
+ * Waits for cuda_stream (steps already queued may read the old schedule).
+ * Without FP8ADAM_FLAG_JIT_EVERY_STEP the schedule starts at step 2 or later:
+ * step 1 takes the amax pre-pass, which the host decides (run it with
+ * fp8adam_step).  If any entry needs the grad-norm pre-pass (loss_scale != 1,
+ * max_norm > 0 or skip_nonfinite), every scheduled step runs it (an entry
+ * without those options gets multiplier 1 and the same results).
+ *
+ * fp8adam_step_scheduled: queues one step on cuda_stream: a one-thread kernel
+ * copies the entry of the device step counter and advances the counter, then
+ * the step's kernels read that entry.  It keeps no per-step state on the host,
+ * so it can be captured once into a CUDA graph and the graph replayed, each
+ * replay the next step.  A step past the end of the schedule updates nothing
+ * and sets the context's error word: fp8adam_check then returns
+ * FP8ADAM_ERR_SCHEDULE_END (and clears it).  The results of each step equal
+ * fp8adam_step_ex with that entry's parameters.  INVALID_ARG without a
+ * schedule.
+ *
+ * fp8adam_get_schedule_step: *next_step = the step the next scheduled step
+ * will run (waits for cuda_stream). */
+int fp8adam_set_schedule(fp8adam_ctx* ctx, const fp8adam_step_params* steps,
+                         int32_t count, void* cuda_stream);
+int fp8adam_step_scheduled(fp8adam_ctx* ctx, void* cuda_stream);
+int fp8adam_get_schedule_step(fp8adam_ctx* ctx, int64_t* next_step,
+                              void* cuda_stream);
 
 /* Results of the last fp8adam_step_ex pre-pass: *grad_norm = the global L2
  * norm of the unscaled gradients, *skipped = 1 if that step was skipped.

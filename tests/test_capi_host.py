@@ -117,6 +117,15 @@ def test_create_rejects_overlapping_written_buffers_on_host(L):
     assert create([t0, (base, base, base, base, 0)]) != capi.ERR_OVERLAP  # an empty tensor has no bytes
 
 
+def test_schedule_entry_points_reject_bad_arguments_on_host(L):
+    sp = (capi.fp8adam_step_params * 1)(capi.fp8adam_step_params(1e-3, 0.9, 0.95, 1e-8, 0.1, 2, 1.0, 0.0, 0))
+    assert L.fp8adam_set_schedule(None, sp, 1, None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_step_scheduled(None, None) == capi.ERR_INVALID_ARG
+    t = ctypes.c_int64(0)
+    assert L.fp8adam_get_schedule_step(None, ctypes.byref(t), None) == capi.ERR_INVALID_ARG
+    assert L.fp8adam_strerror(capi.ERR_SCHEDULE_END).startswith(b"a scheduled step")
+
+
 def test_release_build_has_no_debug_hooks(L):
     assert L.fp8adam_debug_inject_wait(0, 1) == capi.ERR_INVALID_ARG
     assert L.fp8adam_debug_set_numel(None, 0, 0) == capi.ERR_INVALID_ARG
