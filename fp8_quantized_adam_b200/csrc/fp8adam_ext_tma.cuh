@@ -2,7 +2,7 @@
 // fp8adam_step_ex) with its loads staged through shared memory by bulk
 // copies, for FP8 m and v.
 //
-// The pipeline is the default staged step's (tma_stream: 3 x 16 KB stages,
+// The pipeline is the default staged step's (tma_begin / tma_run: 3 x 16 KB stages,
 // one issuing thread, bounded waits, 4 CTAs of 256 threads per SM); the
 // element work adds the options to the default step's:
 //   - the gradient multiplier (loss-scale removal and clipping), one multiply;
@@ -126,21 +126,27 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   if (*(volatile const uint32_t*)err) return;  // an earlier CTA timed out: stop at once
   if (a.skip && *a.skip) return;              // a non-finite gradient: the step is skipped
   if (a.s.cur && !a.s.cur->valid) return;     // the schedule ran out
-  const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
   const Chunk ch = a.s.chunks[blockIdx.x];
   const int ti = ch.tensor;
   FP8ADAM_BOUNDS(ti >= 0 && ti < a.s.num_tensors);
   const TensorDesc td = a.s.tensors[ti];
-  const ExtSeg sg = ext_setup<MF, VF>(a, ti, gm);
   const int64_t e0 = ch.start, e1 = ch.start + ch.len;
   FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
+  // whole sub-tiles are staged when the tensor and its bf16 output (if any)
+  // are 16-byte aligned; the first copies are issued before the set-up below
+  // (multiplier, scales from the amax history, constants)
+  const uint16_t* pb = a.p_bf16 ? a.p_bf16[ti] : nullptr;
+  const bool staged = td.aligned && (pb == nullptr || ((uintptr_t)pb & 15u) == 0);
+  const int nsub = staged ? (int)((e1 - e0) / kSub) : 0;
+  tma_begin(td, e0, nsub, stage, full, abort_flag);
+  const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
+  const ExtSeg sg = ext_setup<MF, VF>(a, ti, gm);
   float am = 0.0f, av = 0.0f;
   uint32_t flushed = 0, sat = 0;
 
   SrChunk su{0u, 0u, 0u};
   if constexpr (SR) su = sr_chunk(a, ti, sg.t_lo, e0 >> 1);
-  const int nsub = ext_vec_ok(td, sg) ? (int)((e1 - e0) / kSub) : 0;
-  if (!tma_stream(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
+  if (!tma_run(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
         ext_consume4<MF, VF, STATS, SR>(a, st, j, td, sg, su, i, am, av, flushed, sat);
       }))
     return;

@@ -135,35 +135,46 @@ __device__ __forceinline__ void consume4(const TmaStage& st, int j, const Tensor
   __stcs(reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(td.v) + i), vq);
 }
 
+// Sub-tile k of the chunk that starts at element e0 of td into stage
+// k % kStages (thread 0 only): arm the stage's barrier with the byte count,
+// then issue the four bulk copies.
+__device__ __forceinline__ void tma_issue(const TensorDesc& td, int64_t e0, int k, TmaStage* stage, uint64_t* full) {
+  TmaStage& st = stage[k % kStages];
+  uint64_t* bar = &full[k % kStages];
+  const int64_t b = e0 + (int64_t)k * kSub;
+  mbar_arrive_expect_tx(bar, (uint32_t)sizeof(TmaStage));
+  if (debug_skip_copies(k)) return;  // debug build: this stage's bytes never arrive
+  bulk_load(st.p, td.p + b, kSub * 4, bar);
+  bulk_load(st.g, td.g + b, kSub * 2, bar);
+  bulk_load(st.m, static_cast<const uint8_t*>(td.m) + b, kSub, bar);
+  bulk_load(st.v, static_cast<const uint8_t*>(td.v) + b, kSub, bar);
+}
+
 // The staged pipeline over the first nsub whole sub-tiles of the chunk that
-// starts at element e0 of td: thread 0 issues the bulk copies of p, g, m, v
-// into the kStages-deep ring, and every thread calls body(st, j, i) for its
-// 2 groups of 4 elements of each sub-tile (stage st, stage offset j, global
-// element i).  `full` and `abort_flag` live in the kernel's shared memory.
-// Returns false if a wait gave up: then bit 0 of *err is set and the copies
+// starts at element e0 of td, in two parts so that a kernel can do its own
+// set-up while the first copies are in flight:
+// - tma_begin initialises the stage barriers and has thread 0 issue the
+//   first kStages sub-tiles;
+// - tma_run then has every thread call body(st, j, i) for its 2 groups of 4
+//   elements of each sub-tile (stage st, stage offset j, global element i),
+//   refilling each stage once all threads are done with it.
+// `full` and `abort_flag` live in the kernel's shared memory.  tma_run
+// returns false if a wait gave up: then bit 0 of *err is set and the copies
 // still in flight have been waited for (bounded), so the CTA can return.
-template <typename Body>
-__device__ __forceinline__ bool tma_stream(const TensorDesc& td, int64_t e0, int nsub, TmaStage* stage,
-                                           uint64_t* full, int& abort_flag, uint32_t* err, Body&& body) {
+__device__ __forceinline__ void tma_begin(const TensorDesc& td, int64_t e0, int nsub, TmaStage* stage,
+                                          uint64_t* full, int& abort_flag) {
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int k = 0; k < kStages && k < nsub; ++k) tma_issue(td, e0, k, stage, full);
   }
   __syncthreads();
-  auto issue = [&](int k) {  // sub-tile k of the chunk into stage k % kStages
-    TmaStage& st = stage[k % kStages];
-    uint64_t* bar = &full[k % kStages];
-    const int64_t b = e0 + (int64_t)k * kSub;
-    mbar_arrive_expect_tx(bar, (uint32_t)sizeof(TmaStage));
-    if (debug_skip_copies(k)) return;  // debug build: this stage's bytes never arrive
-    bulk_load(st.p, td.p + b, kSub * 4, bar);
-    bulk_load(st.g, td.g + b, kSub * 2, bar);
-    bulk_load(st.m, static_cast<const uint8_t*>(td.m) + b, kSub, bar);
-    bulk_load(st.v, static_cast<const uint8_t*>(td.v) + b, kSub, bar);
-  };
-  if (threadIdx.x == 0)
-    for (int k = 0; k < kStages && k < nsub; ++k) issue(k);
+}
+
+template <typename Body>
+__device__ __forceinline__ bool tma_run(const TensorDesc& td, int64_t e0, int nsub, TmaStage* stage,
+                                        uint64_t* full, int& abort_flag, uint32_t* err, Body&& body) {
   for (int k = 0; k < nsub; ++k) {
     const int s = k % kStages;
     if (!mbar_wait(&full[s], (uint32_t)((k / kStages) & 1))) abort_flag = 1;
@@ -185,7 +196,7 @@ __device__ __forceinline__ bool tma_stream(const TensorDesc& td, int64_t e0, int
     __syncthreads();  // every thread is done reading stage s
     if (threadIdx.x == 0 && k + kStages < nsub) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic reads before the async refill
-      issue(k + kStages);
+      tma_issue(td, e0, k + kStages, stage, full);
     }
   }
   return true;
@@ -206,10 +217,15 @@ fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
   const int ti = ch.tensor;
   FP8ADAM_BOUNDS(ti >= 0 && ti < a.num_tensors);
   const TensorDesc td = a.tensors[ti];
-  StepConsts c;
-  if (!step_consts(a, c)) return;
+  if (a.cur && !a.cur->valid) return;  // a scheduled step past the end of its schedule
   const int64_t e0 = ch.start, e1 = ch.start + ch.len;
   FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
+  // whole sub-tiles go through the staged pipeline (aligned tensors only);
+  // the first copies are issued before the per-tensor loads below
+  const int nsub = td.aligned ? (int)((e1 - e0) / kSub) : 0;
+  tma_begin(td, e0, nsub, stage, full, abort_flag);
+  StepConsts c;
+  (void)step_consts(a, c);
   const float s_m = a.scale_m[ti];
   const float s_v = a.scale_v[ti];
   const float s_m_new = pow2scale<MF>(__uint_as_float(a.amax_in_m[ti]), s_m);
@@ -219,9 +235,7 @@ fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
   float am = 0.0f, av = 0.0f;
   uint32_t flushed = 0, sat = 0;
 
-  // whole sub-tiles go through the staged pipeline (aligned tensors only)
-  const int nsub = td.aligned ? (int)((e1 - e0) / kSub) : 0;
-  if (!tma_stream(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
+  if (!tma_run(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
         consume4<MF, VF, STATS>(st, j, td, i, c, inv_s_m, inv_s_v, s_m_new, s_v_new, am, av, flushed, sat);
       }))
     return;
