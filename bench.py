@@ -40,8 +40,8 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum per element of the step kernel,
 # from the ncu capture summarised in profiles/, valid while the kernel sources
 # hash to KERNEL_SHA (null otherwise).
-TRAFFIC_PER_PARAM = 13.4859  # profiles/fp8adam_step_tma_kernel_llama2_100m.md: 876.40 MB + 600.71 MB / 109.53 M
-KERNEL_SHA = "e2bd44da06c55c97"
+TRAFFIC_PER_PARAM = 13.4919  # profiles/fp8adam_step_tma_kernel_llama2_100m.md: 876.44 MB + 601.33 MB / 109.53 M
+KERNEL_SHA = "e478f8f55a5b1dab"
 
 
 def kernel_sha() -> str:
