@@ -71,8 +71,9 @@ def test_learning_rate_schedule_against_the_oracle():
         assert float(M.scale_m[i]) == float(r.scale_m[0]) and float(M.amax_v[i]) == float(r.amax_v[0]), i
 
 
-@pytest.mark.parametrize("opts", [{}, dict(stochastic_rounding=True, seed=5, amax_history_len=4, margin_v=1)],
-                         ids=["default", "sr_history_margin"])
+@pytest.mark.parametrize("opts", [{}, dict(stochastic_rounding=True, seed=5, amax_history_len=4, margin_v=1),
+                                  dict(tma=False), dict(tma=False, stochastic_rounding=True, seed=5, amax_history_len=4)],
+                         ids=["default", "sr_history_margin", "vector", "vector_sr_history"])
 def test_captured_graph_replays_equal_regular_steps(opts):
     """One fp8adam_step_scheduled captured in a CUDA graph, replayed once per
     step with new gradients written between replays, against fp8adam_step_ex
