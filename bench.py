@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -41,14 +42,22 @@ FALLBACK_HBM_GBS = 6650.0
 # from the ncu capture summarised in profiles/, valid while the kernel sources
 # hash to KERNEL_SHA (null otherwise).
 TRAFFIC_PER_PARAM = 13.4919  # profiles/fp8adam_step_tma_kernel_llama2_100m.md: 876.44 MB + 601.33 MB / 109.53 M
-KERNEL_SHA = "e478f8f55a5b1dab"
+KERNEL_SHA = "13c4c231bad67f2b"
+
+
+def _code_only(src: str) -> str:
+    """C++ source without comments and blank runs (the step kernel's code is
+    what the traffic figure was measured for, not its commentary)."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(" ".join(line.split()) for line in src.splitlines() if line.strip())
 
 
 def kernel_sha() -> str:
     h = hashlib.sha256()
     for f in ("fp8adam_step.cuh", "fp8adam_step_tma.cuh", "fp8_codec.cuh"):  # the step kernel's device code
-        with open(os.path.join(ROOT, "fp8_quantized_adam_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "fp8_quantized_adam_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -1,7 +1,9 @@
 // fp8adam_ext.cuh -- optional variants of the FP8-moment AdamW step.
 //
 // These are the options of fp8adam_create_ex / fp8adam_step_ex; the default
-// step (fp8adam_step_kernel) contains none of them.
+// step kernels (fp8adam_step_tma_kernel, fp8adam_step_kernel) contain none of
+// them.  This file has the element code of the options, the per-thread-load
+// variant kernel and the pre-passes; fp8adam_ext_tma.cuh the staged kernel.
 //   - amax history (DelayedScaling "amax_history_len", algo MAX) and margin
 //     ("margin"), from the transformer_engine example of "FP8训练的稳定性挑战…";
 //   - update from the stored (requantised) moments instead of this step's

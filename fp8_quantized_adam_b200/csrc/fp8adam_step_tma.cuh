@@ -9,11 +9,13 @@
 // all threads consume a stage from shared memory (2 x 4 elements each),
 // store p and the new codes straight to global, and release the stage.  The
 // copies run ahead of the arithmetic, so the bytes in flight no longer depend
-// on registers.  4 CTAs of 256 threads per SM (64 registers, 48 KB of shared
-// memory each).  Measured on the 7B-shaped layout: 14.3 ms per step against
-// 14.85 ms for per-thread vector loads and 14.1 ms for a probe with the same
-// copies and no arithmetic; a warp-specialised form (separate producer warp,
-// empty/full barriers) and 1024-element sub-tiles were slower.
+// on registers.  4 CTAs of 256 threads per SM (62-64 registers, 48 KB of
+// shared memory each).  A chunk's first copies are issued before its
+// per-tensor loads and scale arithmetic, which then overlap the fill.
+// Measured on the 7B-shaped layout: 14.15 ms per step against 14.85 ms for
+// per-thread vector loads and 14.1 ms for a probe with the same copies and no
+// arithmetic; a warp-specialised form (separate producer warp, empty/full
+// barriers) and 1024-element sub-tiles were slower.
 //
 // A tensor that is not 16-byte aligned, and the part of a chunk beyond its
 // last whole sub-tile, go through the per-thread path of fp8adam_step.cuh.
