@@ -278,6 +278,22 @@ def test_stress_20k_tensors_full_parity_2_steps():
     assert res["elements"] == workloads.total_params(r.specs)
 
 
+def test_stress_20k_tensors_50_steps_subset():
+    """The stress configuration's 50 steps (20,000 x 4096 + 8 x 2^28, one
+    launch per step); 300 of the small tensors, spread over the list,
+    against the oracle at steps 1, 2, 10, 25 and 50 (tensors are independent,
+    so a subset check is exact), and the scale invariants of every tensor."""
+    specs = workloads.layout("stress_20k")
+    small = [i for i, s in enumerate(specs) if s.numel == 4096]
+    subset = small[::len(small) // 300][:300]
+    r = Run(specs, workloads.CFG_ID["stress_20k"], subset=subset)
+    for t in range(1, 51):
+        r.step(with_oracle=True)
+        if t in (1, 2, 10, 25, 50):
+            r.compare()
+            r.check_invariants()
+
+
 @pytest.mark.slow
 def test_llama2_7b_layout_subset_3_steps():
     specs = workloads.layout("llama2_7b")
