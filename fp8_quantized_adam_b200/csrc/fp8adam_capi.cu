@@ -360,10 +360,10 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
       (opts->amax_history_len > 1 && (!opts->amax_history_m || !opts->amax_history_v)))
     return FP8ADAM_ERR_INVALID_ARG;
 
-  std::vector<TensorDesc> desc((size_t)num_tensors);
   for (int32_t i = 0; i < num_tensors; ++i) {
     const fp8adam_tensor& t = tensors[i];
-    if (t.numel < 0) return FP8ADAM_ERR_INVALID_ARG;
+    // 2^48 elements bounds every size and byte offset computed below far from overflow
+    if (t.numel < 0 || t.numel > ((int64_t)1 << 48)) return FP8ADAM_ERR_INVALID_ARG;
     if (t.numel > 0 && (!t.param || !t.grad || !t.m || !t.v)) return FP8ADAM_ERR_INVALID_ARG;
   }
   // no written buffer (p, m, v, the bf16 copy) may overlap any other buffer
@@ -410,20 +410,27 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
   }
   const int64_t total_units = count_chunks(chunk);
   if (total_units > INT32_MAX / 2) return FP8ADAM_ERR_INVALID_ARG;
+  // the host-side tables (no exception may cross the ABI)
+  std::vector<TensorDesc> desc;
   std::vector<Chunk> chunks;
-  chunks.reserve((size_t)total_units);
-  for (int32_t i = 0; i < num_tensors; ++i) {
-    const fp8adam_tensor& t = tensors[i];
-    TensorDesc& d = desc[(size_t)i];
-    d.p = t.param;
-    d.g = t.grad;
-    d.m = t.m;
-    d.v = t.v;
-    d.numel = t.numel;
-    d.nunits = (int32_t)((t.numel + chunk - 1) / chunk);
-    d.aligned = aligned16(t.param) && aligned16(t.grad) && aligned16(t.m) && aligned16(t.v);
-    for (int64_t st = 0; st < t.numel; st += chunk)
-      chunks.push_back(Chunk{i, (int32_t)(t.numel - st < chunk ? t.numel - st : chunk), st});
+  try {
+    desc.resize((size_t)num_tensors);
+    chunks.reserve((size_t)total_units);
+    for (int32_t i = 0; i < num_tensors; ++i) {
+      const fp8adam_tensor& t = tensors[i];
+      TensorDesc& d = desc[(size_t)i];
+      d.p = t.param;
+      d.g = t.grad;
+      d.m = t.m;
+      d.v = t.v;
+      d.numel = t.numel;
+      d.nunits = (int32_t)((t.numel + chunk - 1) / chunk);
+      d.aligned = aligned16(t.param) && aligned16(t.grad) && aligned16(t.m) && aligned16(t.v);
+      for (int64_t st = 0; st < t.numel; st += chunk)
+        chunks.push_back(Chunk{i, (int32_t)(t.numel - st < chunk ? t.numel - st : chunk), st});
+    }
+  } catch (...) {
+    return FP8ADAM_ERR_OOM;
   }
 
   fp8adam_ctx* c = new (std::nothrow) fp8adam_ctx();
@@ -805,7 +812,11 @@ extern "C" int fp8adam_step_host(fp8adam_ctx* ctx, const fp8adam_step_params* pa
       cudaGetLastError();
       return FP8ADAM_ERR_CUDA;
     }
-    ctx->grp_event.assign((size_t)G, nullptr);
+    try {
+      ctx->grp_event.assign((size_t)G, nullptr);
+    } catch (...) {
+      return FP8ADAM_ERR_OOM;
+    }
     for (int g = 0; g < G; ++g)
       if (cudaEventCreateWithFlags(&ctx->grp_event[(size_t)g], cudaEventDisableTiming) != cudaSuccess) {
         cudaGetLastError();

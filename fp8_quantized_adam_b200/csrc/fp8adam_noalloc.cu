@@ -230,7 +230,7 @@ extern "C" int fp8adam_step_noalloc(const fp8adam_tensor* tensors, int32_t num_t
   int64_t chunks = 0;
   for (int32_t i = 0; i < num_tensors; ++i) {
     const fp8adam_tensor& t = tensors[i];
-    if (t.numel < 0) return FP8ADAM_ERR_INVALID_ARG;
+    if (t.numel < 0 || t.numel > ((int64_t)1 << 48)) return FP8ADAM_ERR_INVALID_ARG;
     if (t.numel > 0 && (!t.param || !t.grad || !t.m || !t.v)) return FP8ADAM_ERR_INVALID_ARG;
     TensorDesc& d = g_host_image.desc[i];
     d.p = t.param;

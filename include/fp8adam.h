@@ -88,7 +88,7 @@ typedef enum {
                                             shared memory with TMA bulk copies. */
 
 /* One tensor.  param: fp32[numel]; grad: bf16[numel] (raw bits); m, v:
- * uint8[numel] codes or fp32[numel] in FP8ADAM_FP32 mode.  Any numel >= 0
+ * uint8[numel] codes or fp32[numel] in FP8ADAM_FP32 mode.  Any numel in [0, 2^48]
  * (an empty tensor is skipped and its state left as is).  Buffers that are
  * 16-byte aligned take the vectorised path; others are processed element by
  * element, with the same results. */
@@ -107,7 +107,7 @@ typedef struct fp8adam_ctx fp8adam_ctx; /* opaque */
  * (host array) to the device, allocates the context's accumulators and
  * synchronises once.  scale_m/scale_v/amax_m/amax_v: device fp32
  * [num_tensors].  m_fmt/v_fmt: fp8adam_fmt.  Returns INVALID_ARG for null
- * pointers, num_tensors < 1 or numel < 0; UNSUPPORTED_FMT; OVERLAP if a
+ * pointers, num_tensors < 1, numel < 0 or > 2^48; UNSUPPORTED_FMT; OVERLAP if a
  * buffer the step writes (param, m, v, and with fp8adam_create_ex the bf16
  * copies) overlaps any other buffer of the list (gradients, which are only
  * read, may overlap one another); OOM; CUDA.  Checked on the host before

@@ -115,6 +115,7 @@ def test_create_rejects_overlapping_written_buffers_on_host(L):
     t4 = (base + 4 * n, base + 0xA0000, base + 0xB0000, base + 0xC0000, n)
     assert create([t0, t4]) != capi.ERR_OVERLAP                       # adjacent, not overlapping
     assert create([t0, (base, base, base, base, 0)]) != capi.ERR_OVERLAP  # an empty tensor has no bytes
+    assert create([(base, base + 8, base + 16, base + 24, (1 << 48) + 1)]) == capi.ERR_INVALID_ARG  # size bound
 
 
 def test_schedule_entry_points_reject_bad_arguments_on_host(L):
