@@ -125,6 +125,12 @@ class FP8AdamW:
             self.ctx = capi.fp8adam_create_ex(arr, T, opts)
         self.device = dev
 
+    def _call(self, fn, *args):
+        """A C ABI call on the optimizer's device (the library requires the
+        device current at create to be current at every call)."""
+        with torch.cuda.device(self.device):
+            return fn(*args)
+
     def step(self, stream: Optional[torch.cuda.Stream] = None, lr: Optional[float] = None,
              loss_scale: float = 1.0, max_norm: float = 0.0, skip_nonfinite: bool = False) -> None:
         """One AdamW step on every tensor, queued on ``stream`` (default: the
@@ -135,12 +141,12 @@ class FP8AdamW:
         self.t += 1
         lr = self.lr if lr is None else lr
         if loss_scale == 1.0 and max_norm <= 0.0 and not skip_nonfinite:
-            capi.fp8adam_step(self.ctx, lr, self.betas[0], self.betas[1], self.eps, self.weight_decay, self.t,
+            self._call(capi.fp8adam_step, self.ctx, lr, self.betas[0], self.betas[1], self.eps, self.weight_decay, self.t,
                               s.cuda_stream)
         else:
             sp = capi.fp8adam_step_params(lr, self.betas[0], self.betas[1], self.eps, self.weight_decay, self.t,
                                           loss_scale, max_norm, 1 if skip_nonfinite else 0)
-            capi.fp8adam_step_ex(self.ctx, sp, s.cuda_stream)
+            self._call(capi.fp8adam_step_ex, self.ctx, sp, s.cuda_stream)
 
     def step_host(self, host_grads: Sequence[torch.Tensor], amax_out: Optional[torch.Tensor] = None,
                   stream: Optional[torch.cuda.Stream] = None, lr: Optional[float] = None,
@@ -172,7 +178,7 @@ class FP8AdamW:
         sp = capi.fp8adam_step_params(lr, self.betas[0], self.betas[1], self.eps, self.weight_decay, self.t,
                                       loss_scale, max_norm, 1 if skip_nonfinite else 0)
         try:
-            capi.fp8adam_step_host(self.ctx, sp, ptrs, out, s.cuda_stream)
+            self._call(capi.fp8adam_step_host, self.ctx, sp, ptrs, out, s.cuda_stream)
         except capi.Fp8AdamError:
             self.t -= 1
             raise
@@ -188,7 +194,7 @@ class FP8AdamW:
                                           first + k, loss_scale, max_norm, 1 if skip_nonfinite else 0)
                  for k, lr in enumerate(lrs)]
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
-        capi.fp8adam_set_schedule(self.ctx, steps, s.cuda_stream)
+        self._call(capi.fp8adam_set_schedule, self.ctx, steps, s.cuda_stream)
 
     def step_scheduled(self, stream: Optional[torch.cuda.Stream] = None) -> None:
         """The next step of the schedule, with no per-step host state: can be
@@ -196,32 +202,32 @@ class FP8AdamW:
         does not follow graph replays; ``scheduled_step()`` reads the device
         counter."""
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
-        capi.fp8adam_step_scheduled(self.ctx, s.cuda_stream)
+        self._call(capi.fp8adam_step_scheduled, self.ctx, s.cuda_stream)
         self.t += 1
 
     def scheduled_step(self, stream: Optional[torch.cuda.Stream] = None) -> int:
         """The step the next scheduled step will run (synchronises the stream)."""
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
-        return capi.fp8adam_get_schedule_step(self.ctx, s.cuda_stream)
+        return self._call(capi.fp8adam_get_schedule_step, self.ctx, s.cuda_stream)
 
     def grad_info(self, stream: Optional[torch.cuda.Stream] = None):
         """(global grad L2 norm, skipped) of the last step with a gradient
         pre-pass (synchronises the stream)."""
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
-        return capi.fp8adam_get_grad_info(self.ctx, s.cuda_stream)
+        return self._call(capi.fp8adam_get_grad_info, self.ctx, s.cuda_stream)
 
     def check(self, stream: Optional[torch.cuda.Stream] = None) -> None:
         """Raise if a kernel's bounded wait ran out (synchronises the stream)."""
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
-        capi.fp8adam_check(self.ctx, s.cuda_stream)
+        self._call(capi.fp8adam_check, self.ctx, s.cuda_stream)
 
     def stats(self, stream: Optional[torch.cuda.Stream] = None):
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
-        return capi.fp8adam_get_stats(self.ctx, s.cuda_stream)
+        return self._call(capi.fp8adam_get_stats, self.ctx, s.cuda_stream)
 
     def reset_stats(self, stream: Optional[torch.cuda.Stream] = None) -> None:
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
-        capi.fp8adam_reset_stats(self.ctx, s.cuda_stream)
+        self._call(capi.fp8adam_reset_stats, self.ctx, s.cuda_stream)
 
     # ---- checkpoint / resume ------------------------------------------
     def state_dict(self) -> dict:
@@ -252,7 +258,7 @@ class FP8AdamW:
 
     def close(self) -> None:
         if getattr(self, "ctx", None):
-            capi.fp8adam_destroy(self.ctx)
+            self._call(capi.fp8adam_destroy, self.ctx)
             self.ctx = None
 
     def __del__(self):  # pragma: no cover - best effort

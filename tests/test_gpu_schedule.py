@@ -93,7 +93,7 @@ def test_captured_graph_replays_equal_regular_steps(opts):
     side.wait_stream(s)
     with torch.cuda.stream(side):
         with torch.cuda.graph(graph, stream=side):
-            capi.fp8adam_step_scheduled(b.opt.ctx, side.cuda_stream)
+            b.opt.step_scheduled(stream=side)  # the binding's call, device guard included
     s.wait_stream(side)
     torch.cuda.synchronize()
     assert b.opt.scheduled_step() == 2  # capture ran nothing
