@@ -1,4 +1,4 @@
-"""ZeRO-1 orchestration with world_size 2 on gloo (CPU).
+"""ZeRO-1 orchestration with world_size 2 and 3 on gloo (CPU).
 
 The sharded step's bookkeeping is what is tested here: the whole-tensor
 partition, rank-blocked flat buffers, reduce-scatter of the gradients,
@@ -11,6 +11,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.multiprocessing as mp
 
@@ -75,7 +76,7 @@ def _worker(rank, world, port, q):
         ok = all((v.numpy().view(np.uint32) == st.p.view(np.uint32)).all() for v, st in zip(L.views(params), ref))
         q.put(("rank0", ok, [len(p) for p in L.parts]))
     else:
-        q.put(("rank1", True, None))
+        q.put(("rank%d" % rank, True, None))
     ranks.finish()
 
 
@@ -85,19 +86,20 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_zero1_world2_matches_single_process_oracle():
+@pytest.mark.parametrize("world", [2, 3])
+def test_zero1_matches_single_process_oracle(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    ps = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    ps = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in ps:
         p.start()
-    res = dict((k, (ok, parts)) for k, ok, parts in (q.get(timeout=300), q.get(timeout=300)))
+    res = dict((k, (ok, parts)) for k, ok, parts in (q.get(timeout=300) for _ in range(world)))
     for p in ps:
         p.join(timeout=120)
     ok, parts = res["rank0"]
-    assert ok
-    assert sum(parts) == len(SIZES) and min(parts) >= 1  # both ranks own tensors
+    assert ok and all(res["rank%d" % r][0] for r in range(1, world))
+    assert sum(parts) == len(SIZES) and min(parts) >= 1  # every rank owns tensors
 
 
 def test_shard_layout_blocks():
