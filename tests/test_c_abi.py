@@ -78,3 +78,14 @@ def test_c_example_matches_the_oracle(tmp_path):
     for i in range(2):
         assert state[0 + i] == ref[i].scale_m[0] and state[2 + i] == ref[i].scale_v[0]
         assert state[4 + i] == ref[i].amax_m[0] and state[6 + i] == ref[i].amax_v[0]
+
+
+def test_header_compiles_as_cpp(tmp_path):
+    """The header's extern "C" guard: a C++ translation unit sees C linkage."""
+    src = tmp_path / "use.cpp"
+    src.write_text('#include "fp8adam.h"\n'
+                   'extern "C" int fp8adam_step(fp8adam_ctx*, float, float, float, float, float, int64_t, void*);\n'
+                   'int main() { return fp8adam_strerror(FP8ADAM_OK) ? 0 : 1; }\n')
+    r = subprocess.run(["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-I",
+                        os.path.join(ROOT, "include"), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
