@@ -153,12 +153,92 @@ def test_grad_sumsq_is_the_exact_sum(orc):
     assert s == float(exact)  # Fraction -> float rounds to nearest even
 
 
-def test_grad_multiplier_closed_form(orc):
-    for sumsq, S, mx in ((4.0, 1.0, 1.0), (400.0, 1.0, 1.0), (9e6, 1024.0, 1.0), (0.0, 8.0, 1.0),
-                         (1e4, 2.0, 0.0), (2.5e-3, 65536.0, 0.5)):
-        inv = 1.0 / S
-        coef = 1.0 if mx <= 0 else min(1.0, mx / (math.sqrt(sumsq) * inv + 1e-6))
-        assert orc.grad_multiplier(sumsq, S, mx) == f32(inv * coef)
+def _torch_amp_multiplier(grad_bits, loss_scale, max_norm):
+    """The factor torch's mixed-precision recipe applies to the scaled
+    gradients: unscale (divide by the loss scale), then
+    torch.nn.utils.clip_grad_norm_(params, max_norm) -- the routine printed
+    in the clip_grad_norm_ example of "FP8训练的稳定性挑战…" ("梯度裁剪") --
+    all in float64.  max_norm <= 0 means no clipping (max_norm = inf for
+    torch).  The factor is read back from the clipped gradients: the
+    clipping coefficient is g_clipped / g_unscaled for a non-zero element,
+    and the multiplier of the scaled gradients is that coefficient / S."""
+    params, unscaled = [], []
+    for bits in grad_bits:
+        g = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).double()
+        p = torch.zeros(g.numel(), dtype=torch.float64, requires_grad=True)
+        p.grad = g / float(loss_scale)
+        params.append(p)
+        unscaled.append(p.grad.clone())
+    torch.nn.utils.clip_grad_norm_(params, max_norm if max_norm > 0 else float("inf"))
+    for p, u in zip(params, unscaled):
+        nz = torch.nonzero(u)
+        if len(nz):
+            k = int(nz[0, 0])
+            coef = float(p.grad[k]) / float(u[k])
+            return coef / float(loss_scale), math.sqrt(sum(float((x * x).sum()) for x in unscaled))
+    return 1.0 / float(loss_scale), 0.0
+
+
+def _ulp32(x):
+    x = abs(f32(x))
+    return float(np.spacing(np.float32(x)))
+
+
+def test_grad_multiplier_matches_torch_clip_grad_norm(orc):
+    """The oracle's multiplier c = (1/S)*min(1, max_norm/(norm+1e-6)) with
+    norm the L2 norm of the unscaled gradients, against torch's own
+    unscale + clip_grad_norm_ on the same bf16 gradients: c must be torch's
+    float64 factor rounded to fp32 (a tie band of 1e-9 of half an ulp
+    allows for torch's own float64 rounding).  The cases cover several loss
+    scales (powers of two and not), clipping off, norms on both sides of
+    max_norm, max_norm within an fp32 ulp of the norm, and norms so small
+    that the 1e-6 in the denominator decides the result."""
+    rng = np.random.default_rng(77)
+    sets = []
+    for scale_exp, n_tensors in ((-3, 3), (-6, 2), (0, 4), (-9, 1)):
+        sets.append([_bf16_bits(rng.standard_normal(int(rng.integers(1, 5000))) * 10.0 ** (scale_exp +
+                     rng.uniform(-1, 1))) for _ in range(n_tensors)])
+    cases = 0
+    for grads in sets:
+        sumsq, bad = orc.grad_sumsq(grads)
+        assert bad == 0
+        for S in (1.0, 2.0, 1024.0, 65536.0, 1000.0, 3.0):
+            _, norm = _torch_amp_multiplier(grads, S, 0.0)
+            maxes = [0.0, -1.0, 1.0, 0.5, 100.0, 1e-6, norm * 2.0, norm * 0.5]
+            nf = f32(norm)
+            maxes += [nf, float(np.nextafter(np.float32(nf), np.float32(0))),
+                      float(np.nextafter(np.float32(nf), np.float32(np.inf)))]
+            for mx in maxes:
+                mx = f32(mx)
+                c_ref, _ = _torch_amp_multiplier(grads, S, mx)
+                c = orc.grad_multiplier(sumsq, S, mx)
+                assert abs(c - c_ref) <= 0.5 * _ulp32(c) * (1 + 1e-9), (S, mx, norm, c, c_ref)
+                cases += 1
+    assert cases == 4 * 6 * 11
+
+
+def test_grad_multiplier_distinguishes_plausible_mistakes(orc):
+    """The torch pin above would catch each of these mistakes of the
+    formula: the norm of the scaled instead of the unscaled gradients, the
+    1e-6 dropped or multiplied in, and the clamp to 1 missing."""
+    caught = {"scaled norm": False, "no eps": False, "eps times norm": False, "no clamp": False}
+    for val, S, mx in ((1e-7, 1024.0, 1e-6), (1e-7, 1.0, 1e-6), (1e-3, 1.0, 100.0), (0.25, 4.0, 1.0)):
+        grads = [_bf16_bits(np.full(100, val, np.float32))]
+        sumsq, _ = orc.grad_sumsq(grads)
+        c_ref, _ = _torch_amp_multiplier(grads, S, mx)
+        c = orc.grad_multiplier(sumsq, S, mx)
+        assert abs(c - c_ref) <= 0.5 * _ulp32(c) * (1 + 1e-9)
+        norm = math.sqrt(sumsq) / S
+        wrong = {
+            "scaled norm": (1 / S) * min(1.0, mx / (math.sqrt(sumsq) + 1e-6)),
+            "no eps": (1 / S) * min(1.0, mx / norm),
+            "eps times norm": (1 / S) * min(1.0, mx / (norm * (1 + 1e-6))),
+            "no clamp": (1 / S) * mx / (norm + 1e-6),
+        }
+        for k, w in wrong.items():
+            if abs(f32(w) - c_ref) > _ulp32(c_ref):
+                caught[k] = True
+    assert all(caught.values()), caught
 
 
 # ------------------------------------------------------------------ the extended step
