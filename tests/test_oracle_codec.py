@@ -73,8 +73,14 @@ def test_ties_and_saturation(orc):
     # 2^-17 = half of 2^-16 -> 0; 3*2^-17 -> tie between 1 and 2 -> 2;
     # 1.125 midpoint of 1.0 (0x3C) and 1.25 (0x3D) -> 0x3C; 1.375 -> 0x3E
     assert orc.encode(E5, y).tolist() == [0x7B, 0x7B, 0x7B, 0x00, 0x02, 0x3C, 0x3E]
-    assert orc.encode(E4, np.array([np.nan], np.float32))[0] == 0x7F
-    assert orc.encode(E5, np.array([np.nan], np.float32))[0] == 0x7F
+    # NaN of either sign and any payload -> 0x7F in both formats.  The pages
+    # are silent on the sign of a NaN code; this reading follows the B200's
+    # cvt.rn.satfinite conversion, which the exhaustive device test checks on
+    # every NaN input (torch's CPU cast would keep the sign: 0xFF for -NaN)
+    nans = np.array([0x7FC00000, 0xFFC00000, 0x7F800001, 0xFF800001, 0x7FFFFFFF, 0xFFFFFFFF],
+                    np.uint32).view(np.float32)
+    assert (orc.encode(E4, nans) == 0x7F).all() and (orc.encode(E5, nans) == 0x7F).all()
+    assert all(orc.encode_sr(f, float(x), r) == 0x7F for f in (E4, E5) for x in nans for r in (0, 2 ** 32 - 1))
 
 
 def test_worked_example_from_the_pages(orc):
