@@ -17,6 +17,7 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -45,12 +46,36 @@ constexpr size_t kScratchBytes = round256(kAccOff + sizeof(uint32_t) * kAccWords
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 // Host-side image of the tensor table and chunk offsets, copied into the
-// scratch by every call (static storage, not an allocation).
+// scratch by every call, and the byte ranges of the overlap check (static
+// storage, not an allocation).
 struct HostImage {
   TensorDesc desc[kMaxT];
   int32_t begin[kMaxT + 1];
 };
 static HostImage g_host_image;
+
+struct ByteRange {
+  uintptr_t begin, end;
+  bool written;
+};
+static ByteRange g_ranges[4 * kMaxT];
+
+// True if two of the n byte ranges overlap and at least one of them is
+// written (param, m and v are written, grad is read).  Sorted by start in
+// place (std::sort allocates nothing), a range overlaps an earlier one iff
+// it starts before the furthest end seen so far: of any range if it is
+// written, of the written ranges if it is only read.
+bool written_range_overlaps(ByteRange* r, size_t n) {
+  std::sort(r, r + n, [](const ByteRange& a, const ByteRange& b) { return a.begin < b.begin; });
+  uintptr_t end_all = 0, end_written = 0;
+  for (size_t k = 0; k < n; ++k) {
+    const ByteRange& x = r[k];
+    if (x.begin < (x.written ? end_all : end_written)) return true;
+    end_all = end_all > x.end ? end_all : x.end;
+    if (x.written) end_written = end_written > x.end ? end_written : x.end;
+  }
+  return false;
+}
 
 constexpr int kMaxDevices = 64;
 std::atomic<void*> g_scratch_ptr[kMaxDevices];
@@ -116,7 +141,8 @@ __global__ void __launch_bounds__(kThreads) noalloc_kernel(const NoAllocArgs a) 
   }
   const float inv_s_m = __fdiv_rn(1.0f, s_m);
   const float inv_s_v = __fdiv_rn(1.0f, s_v);
-  uint32_t am = 0, av = 0, unused_f = 0, unused_s = 0;
+  float am = 0.0f, av = 0.0f;  // NaN-keeping max, as the regular step kernels reduce it
+  uint32_t unused_f = 0, unused_s = 0;
   const int64_t end = start + len;
   int64_t scalar_from = start;
 
@@ -145,8 +171,8 @@ __global__ void __launch_bounds__(kThreads) noalloc_kernel(const NoAllocArgs a) 
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           moments(c, g[j], mo[j], vo[j], mn[j], vn[j]);
-          am = fp8adam::umax(am, abs_bits(mn[j]));
-          av = fp8adam::umax(av, abs_bits(vn[j]));
+          am = fmax_nan(am, fabsf(mn[j]));
+          av = fmax_nan(av, fabsf(vn[j]));
         }
         if constexpr (WRITE) {
           float pk[4] = {pv[k].x, pv[k].y, pv[k].z, pv[k].w};
@@ -170,8 +196,8 @@ __global__ void __launch_bounds__(kThreads) noalloc_kernel(const NoAllocArgs a) 
     const float g = __uint_as_float((uint32_t)td.g[i] << 16);
     float mn, vn;
     moments(c, g, load1<MF>(td.m, i, inv_s_m), load1<VF>(td.v, i, inv_s_v), mn, vn);
-    am = fp8adam::umax(am, abs_bits(mn));
-    av = fp8adam::umax(av, abs_bits(vn));
+    am = fmax_nan(am, fabsf(mn));
+    av = fmax_nan(av, fabsf(vn));
     if constexpr (WRITE) {
       td.p[i] = update(c, td.p[i], mn, vn);
       store1<MF, false, false>(td.m, i, mn, s_m_new, unused_f, unused_s);
@@ -179,8 +205,8 @@ __global__ void __launch_bounds__(kThreads) noalloc_kernel(const NoAllocArgs a) 
     }
   }
 
-  const uint32_t bm = block_max(am, red[0]);
-  const uint32_t bv = block_max(av, red[1]);
+  const uint32_t bm = block_max(__float_as_uint(am), red[0]);
+  const uint32_t bv = block_max(__float_as_uint(av), red[1]);
   if (threadIdx.x == 0) {
     if (bm) atomicMax(a.acc_m + ti, bm);
     if (bv) atomicMax(a.acc_v + ti, bv);
@@ -247,6 +273,22 @@ extern "C" int fp8adam_step_noalloc(const fp8adam_tensor* tensors, int32_t num_t
     if (chunks > INT32_MAX) return FP8ADAM_ERR_INVALID_ARG;
   }
   g_host_image.begin[num_tensors] = (int32_t)chunks;
+
+  // as fp8adam_create: no written buffer (p, m, v) may overlap another buffer
+  {
+    const size_t mb = m_fmt == FP8ADAM_FP32 ? 4 : 1, vb = v_fmt == FP8ADAM_FP32 ? 4 : 1;
+    size_t nr = 0;
+    for (int32_t i = 0; i < num_tensors; ++i) {
+      const fp8adam_tensor& t = tensors[i];
+      if (t.numel == 0) continue;
+      const size_t n = (size_t)t.numel;
+      g_ranges[nr++] = ByteRange{(uintptr_t)t.param, (uintptr_t)t.param + 4 * n, true};
+      g_ranges[nr++] = ByteRange{(uintptr_t)t.grad, (uintptr_t)t.grad + 2 * n, false};
+      g_ranges[nr++] = ByteRange{(uintptr_t)t.m, (uintptr_t)t.m + mb * n, true};
+      g_ranges[nr++] = ByteRange{(uintptr_t)t.v, (uintptr_t)t.v + vb * n, true};
+    }
+    if (written_range_overlaps(g_ranges, nr)) return FP8ADAM_ERR_OVERLAP;
+  }
 
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return FP8ADAM_ERR_CUDA;
