@@ -543,8 +543,15 @@ static bool valid_hparams(float lr, float beta1, float beta2, float eps, float w
          beta2 >= 0.0f && beta2 < 1.0f && eps >= 0.0f && std::isfinite(eps);
 }
 
+// The grad-norm pre-pass is needed for clipping (the global norm) and for
+// skip-on-non-finite (the non-finite count).  A loss scale alone is a
+// constant multiplier, 1/loss_scale, computed on the host as the pre-pass's
+// finalize kernel computes it without clipping (double, rounded once).
 static bool needs_prepass(const fp8adam_step_params& p) {
-  return p.loss_scale != 1.0f || p.max_norm > 0.0f || p.skip_nonfinite != 0;
+  return p.max_norm > 0.0f || p.skip_nonfinite != 0;
+}
+static float host_multiplier(const fp8adam_step_params& p) {
+  return (float)(1.0 / (double)p.loss_scale);
 }
 
 // The step over chunks [c0, c1) of the chunk table: every chunk of the
@@ -559,7 +566,7 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
                           bool first, const SchedEntry* cur = nullptr) {
   if (c1 <= c0) return FP8ADAM_OK;  // only empty tensors
   const bool prepass = cur ? ctx->sched_prepass : needs_prepass(p);
-  const bool ext = ctx->ext || prepass;
+  const bool ext = ctx->ext || prepass || (!cur && p.loss_scale != 1.0f);
 
   StepArgs a;
   a.c = make_consts(p);
@@ -623,6 +630,7 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
     e.sr_key[r][1] = (uint32_t)(ctx->seed >> 32) + (uint32_t)r * 0xBB67AE85u;
   }
   e.t_lo = (uint32_t)p.step;
+  e.gm_const = cur ? 1.0f : host_multiplier(p);
   e.grad_mult = nullptr;
   e.skip = nullptr;
   e.p_bf16 = ctx->d_bf16;
@@ -729,7 +737,9 @@ extern "C" int fp8adam_set_schedule(fp8adam_ctx* ctx, const fp8adam_step_params*
     e.t_lo = (uint32_t)p.step;
     e.hist_slot = ctx->hist_len ? (int32_t)((p.step - 1) % ctx->hist_len) : 0;
     e.valid = 1;
-    prepass = prepass || needs_prepass(p);
+    // a scheduled step reads its loss scale from the entry, so any scale
+    // other than 1 takes the pre-pass (whose finalize kernel reads it)
+    prepass = prepass || needs_prepass(p) || p.loss_scale != 1.0f;
   }
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return FP8ADAM_ERR_CUDA;

@@ -42,7 +42,8 @@ struct ExtArgs {
   float* hist_v;
   uint32_t sr_key[10][2];    // Philox round keys: round r uses seed + r * (0x9E3779B9, 0xBB67AE85)
   uint32_t t_lo;             // the step (counter word 3)
-  const float* grad_mult;   // device scalar, or null (1.0)
+  const float* grad_mult;   // device scalar from the grad-norm pre-pass, or null (then gm_const)
+  float gm_const;           // gradient multiplier without a pre-pass: 1/loss_scale (1.0: none)
   const uint32_t* skip;     // device flag, or null
   uint16_t* const* p_bf16;  // device array [T] of bf16 outputs (entries may be null), or null
 };
@@ -383,7 +384,7 @@ fp8adam_step_ext_kernel(const ExtArgs a) {
   __shared__ uint32_t red[4][kThreads / 32];
   if (a.skip && *a.skip) return;  // a non-finite gradient: the step is skipped
   if (a.s.cur && !a.s.cur->valid) return;  // the schedule ran out
-  const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
+  const float gm = a.grad_mult ? *a.grad_mult : a.gm_const;
   const Chunk ch = a.s.chunks[blockIdx.x];
   const int ti = ch.tensor;
   FP8ADAM_BOUNDS(ti >= 0 && ti < a.s.num_tensors);
@@ -408,7 +409,7 @@ fp8adam_amax_ext_kernel(const ExtArgs a) {
   const StepArgs& S = a.s;
   StepConsts c;
   if (!step_consts(S, c)) return;
-  const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
+  const float gm = a.grad_mult ? *a.grad_mult : a.gm_const;
   const Chunk ch = S.chunks[blockIdx.x];
   const int ti = ch.tensor;
   FP8ADAM_BOUNDS(ti >= 0 && ti < S.num_tensors);

@@ -5,7 +5,9 @@
 // The pipeline is the default staged step's (tma_begin / tma_run: 3 x 16 KB stages,
 // one issuing thread, bounded waits, 4 CTAs of 256 threads per SM); the
 // element work adds the options to the default step's:
-//   - the gradient multiplier (loss-scale removal and clipping), one multiply;
+//   - the gradient multiplier (loss-scale removal and clipping: from the
+//     grad-norm pre-pass, or a host constant 1/loss_scale without one), one
+//     multiply;
 //   - the encode scales from the amax history and the margin (per chunk);
 //   - stochastic rounding (a compile-time switch: Philox4x32-10 words for two
 //     elements per call, and the integer SR encoder), or round-to-nearest
@@ -139,7 +141,7 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   const bool staged = td.aligned && (pb == nullptr || ((uintptr_t)pb & 15u) == 0);
   const int nsub = staged ? (int)((e1 - e0) / kSub) : 0;
   tma_begin(td, e0, nsub, stage, full, abort_flag);
-  const float gm = a.grad_mult ? *a.grad_mult : 1.0f;
+  const float gm = a.grad_mult ? *a.grad_mult : a.gm_const;
   const ExtSeg sg = ext_setup<MF, VF>(a, ti, gm);
   float am = 0.0f, av = 0.0f;
   uint32_t flushed = 0, sat = 0;

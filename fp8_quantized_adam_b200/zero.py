@@ -9,8 +9,13 @@ AdamW.  Each rank holds the full params (fp32) and its own full gradients
      summed gradients of the tensors it owns;
   2. the FP8-moment AdamW step (the CUDA kernels) on the owned tensors only,
      with the 1/world average folded into the kernel as its gradient
-     multiplier (``loss_scale = world``);
-  3. all-gather of the updated params (NCCL), so every rank has them all.
+     multiplier (``loss_scale = world``: a constant kernel argument, no
+     gradient pre-pass unless clipping or skip-on-non-finite is asked for);
+  3. all-gather of the updated params (NCCL), in place: each rank's block of
+     the flat param buffer is its input, so nothing is copied first.
+
+The gradients are reduced in their own dtype, bf16, as NCCL sums the buffer
+it is given: the step's input is the reduced bf16 gradient.
 
 Tensors are assigned whole to ranks (largest first onto the least-loaded rank),
 so a tensor's amax and scale never cross ranks.  For the collectives the flat
@@ -61,16 +66,48 @@ class ShardLayout:
         return [block[self.offset[i]:self.offset[i] + self.numels[i]] for i in self.parts[rank]]
 
 
+class TorchCollectives:
+    """Reduce-scatter (sum) and all-gather through torch.distributed on the
+    tensors' own device: NCCL for CUDA tensors."""
+
+    def __init__(self, group=None):
+        self.group = group
+
+    def reduce_scatter(self, out: torch.Tensor, inp: torch.Tensor) -> None:
+        dist.reduce_scatter_tensor(out, inp, op=dist.ReduceOp.SUM, group=self.group)
+
+    def all_gather(self, out: torch.Tensor, inp: torch.Tensor) -> None:
+        dist.all_gather_into_tensor(out, inp, group=self.group)
+
+
+class HostCollectives(TorchCollectives):
+    """The same collectives through host copies, for a process group without
+    device collectives (gloo): device -> host, the collective on the host
+    buffers, host -> device."""
+
+    def reduce_scatter(self, out: torch.Tensor, inp: torch.Tensor) -> None:
+        h_out = torch.empty(out.shape, dtype=out.dtype)
+        dist.reduce_scatter_tensor(h_out, inp.cpu(), op=dist.ReduceOp.SUM, group=self.group)
+        out.copy_(h_out)
+
+    def all_gather(self, out: torch.Tensor, inp: torch.Tensor) -> None:
+        h_out = torch.empty(out.shape, dtype=out.dtype)
+        dist.all_gather_into_tensor(h_out, inp.cpu(), group=self.group)
+        out.copy_(h_out)
+
+
 class ZeroFP8AdamW:
     """ZeRO-1 FP8-moment AdamW.  ``params`` (fp32) and ``grads`` (bf16) are
     the rank-blocked flat buffers of a ShardLayout (``layout.views`` gives the
     per-tensor views a model would use).  ``local_step`` builds the optimizer
-    of the owned shard; by default the CUDA FP8AdamW."""
+    of the owned shard; by default the CUDA FP8AdamW.  ``collectives``:
+    TorchCollectives (the default: NCCL on CUDA tensors) or HostCollectives."""
 
     def __init__(self, layout: ShardLayout, params: torch.Tensor, grads: torch.Tensor, *,
-                 group=None, make_local: Optional[Callable] = None, **opt_kw):
+                 group=None, make_local: Optional[Callable] = None, collectives=None, **opt_kw):
         self.layout = layout
         self.group = group
+        self.comm = collectives if collectives is not None else TorchCollectives(group)
         self.world = layout.world
         self.rank = dist.get_rank(group) if dist.is_initialized() else 0
         if params.numel() != layout.total or grads.numel() != layout.total:
@@ -91,7 +128,7 @@ class ZeroFP8AdamW:
     def step(self, **step_kw) -> None:
         # 1. summed gradients of the owned tensors
         if self.world > 1:
-            dist.reduce_scatter_tensor(self.g_block, self.grads, op=dist.ReduceOp.SUM, group=self.group)
+            self.comm.reduce_scatter(self.g_block, self.grads)
         else:
             self.g_block.copy_(self.grads)
         # 2. the step on the shard; the average over ranks rides on the
@@ -99,9 +136,10 @@ class ZeroFP8AdamW:
         if self.local is not None:
             ls = float(step_kw.pop("loss_scale", 1.0)) * self.world
             self.local.step(loss_scale=ls, **step_kw)
-        # 3. every rank gets every updated param
+        # 3. every rank gets every updated param; the input is this rank's
+        #    block of the output (NCCL's in-place form)
         if self.world > 1:
-            dist.all_gather_into_tensor(self.params, self.p_block.clone(), group=self.group)
+            self.comm.all_gather(self.params, self.p_block)
 
     def close(self) -> None:
         if self.local is not None and hasattr(self.local, "close"):

@@ -68,7 +68,7 @@ extern "C" {
 #define FP8ADAM_ERR_NOALLOC_LIMIT (-6)   /* more tensors than fp8adam_step_noalloc holds */
 #define FP8ADAM_ERR_DEVICE_TIMEOUT (-7)  /* a kernel's bounded wait ran out (see fp8adam_check) */
 #define FP8ADAM_ERR_DEBUG_BOUNDS (-8)    /* debug build: an access outside its tensor was skipped */
-#define FP8ADAM_ERR_OVERLAP (-9)         /* create: a written buffer overlaps another buffer */
+#define FP8ADAM_ERR_OVERLAP (-9)         /* create, step_noalloc: a written buffer overlaps another */
 #define FP8ADAM_ERR_SCHEDULE_END (-10)   /* a scheduled step ran past its schedule (see fp8adam_check) */
 
 /* Storage format of a moment. */
@@ -227,12 +227,14 @@ typedef struct {
                                 leaves every buffer untouched */
 } fp8adam_step_params;
 
-/* One step with per-step gradient handling.  When loss_scale != 1, max_norm >
- * 0 or skip_nonfinite is set, a pre-pass over all gradients computes (in a
- * fixed reduction order) sumsq = sum of g^2, the multiplier c = (1/loss_scale)
- * * min(1, max_norm / (sqrt(sumsq)/loss_scale + 1e-6)) (double, rounded once
- * to fp32; clip_grad_norm_'s formula) and the non-finite count; the step then
- * uses g*c in place of g.  Asynchronous on cuda_stream. */
+/* One step with per-step gradient handling.  When max_norm > 0 or
+ * skip_nonfinite is set, a pre-pass over all gradients computes (in a fixed
+ * reduction order) sumsq = sum of g^2, the multiplier c = (1/loss_scale) *
+ * min(1, max_norm / (sqrt(sumsq)/loss_scale + 1e-6)) (double, rounded once to
+ * fp32; clip_grad_norm_'s formula) and the non-finite count; the step then
+ * uses g*c in place of g.  With only loss_scale != 1 there is no pre-pass: c =
+ * 1/loss_scale (double, rounded once to fp32; the same value) is a kernel
+ * argument.  Asynchronous on cuda_stream. */
 int fp8adam_step_ex(fp8adam_ctx* ctx, const fp8adam_step_params* params,
                     void* cuda_stream);
 
@@ -245,9 +247,8 @@ int fp8adam_step_ex(fp8adam_ctx* ctx, const fp8adam_step_params* params,
  * waits for the work already queued on cuda_stream.  The tensors are taken in
  * up to 8 groups of about equal size, cut at tensor boundaries; the step of a
  * group is queued on cuda_stream behind that group's copies only, so the
- * copies of later groups overlap it.  With loss_scale != 1, max_norm > 0 or
- * skip_nonfinite the step waits for all copies (the global norm needs every
- * gradient).  amax_host (optional, host float [2 * num_tensors], pinned for
+ * copies of later groups overlap it.  With max_norm > 0 or skip_nonfinite
+ * the step waits for all copies (the global norm needs every gradient).  amax_host (optional, host float [2 * num_tensors], pinned for
  * an asynchronous copy): receives amax_m then amax_v of this step.
  * Asynchronous: host buffers must stay valid, and amax_host is written, only
  * once the work queued on cuda_stream has completed.  The results equal
@@ -354,7 +355,10 @@ uint64_t fp8adam_launch_count(void);
  * be 0 or FP8ADAM_FLAG_JIT_EVERY_STEP (no statistics).
  *
  * - num_tensors > FP8ADAM_NOALLOC_MAX_TENSORS returns FP8ADAM_ERR_NOALLOC_LIMIT
- *   with nothing queued; other argument errors as fp8adam_create/step.
+ *   with nothing queued; other argument errors as fp8adam_create/step,
+ *   overlapping written buffers (FP8ADAM_ERR_OVERLAP) included.
+ * - A NaN moment gives the canonical NaN amax (bits 0x7FFFFFFF), as the
+ *   regular step does.
  * - The first call on a device looks up the scratch array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.

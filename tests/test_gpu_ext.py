@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from fp8_quantized_adam_b200 import FP8AdamW, workloads
+from fp8_quantized_adam_b200 import FP8AdamW, capi, workloads
 from gpu_harness import HP, bf16_host_bits
 
 pytestmark = pytest.mark.gpu
@@ -145,6 +145,21 @@ def test_loss_scale_clip_and_skip(tma):
     r.compare()
     assert r.opt.grad_info()[1] == 1
     assert torch.equal(before, r.M.p)
+
+
+@pytest.mark.parametrize("tma", [True, False], ids=["staged", "vector"])
+def test_loss_scale_alone_runs_no_prepass(tma):
+    """A loss scale without clipping or skipping (as ZeRO-1's 1/world
+    average): the multiplier 1/loss_scale is a kernel argument, so no
+    grad-norm pre-pass runs (one launch per step after step 1's amax
+    pre-pass), and the results equal the oracle's with the pinned multiplier,
+    for power-of-two scales and others."""
+    r = ExtRun(48, tma=tma)
+    for t, ls in enumerate((1024.0, 3.0, 65536.0, 1000.0), start=1):
+        before = capi.fp8adam_launch_count()
+        r.step(loss_scale=ls)
+        assert capi.fp8adam_launch_count() - before == (2 if t == 1 else 1), t
+        r.compare()
 
 
 def test_prepass_only_equals_default_kernel():
