@@ -38,11 +38,12 @@ UNIT = "params/s"
 BYTES_PER_PARAM = 14  # read p 4 + g 2 + m 1 + v 1, write p 4 + m 1 + v 1
 FALLBACK_HBM_GBS = 6650.0
 
-# dram__bytes_read.sum + dram__bytes_write.sum per element of the step kernel,
-# from the ncu capture summarised in profiles/, valid while the kernel sources
-# hash to KERNEL_SHA (null otherwise).
-TRAFFIC_PER_PARAM = 13.4919  # profiles/fp8adam_step_tma_kernel_llama2_100m.md: 876.44 MB + 601.33 MB / 109.53 M
-KERNEL_SHA = "13c4c231bad67f2b"
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per element of the
+# step kernel, from an ncu capture of one launch on a layout far larger than
+# L2, valid while the kernel's device code hashes to KERNEL_SHA (null
+# otherwise).  Null until a capture of the current kernel exists.
+TRAFFIC_PER_PARAM = None
+KERNEL_SHA = None
 
 
 def _code_only(src: str) -> str:
@@ -125,15 +126,44 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- oracle leg
+SINGLE_THREAD_PARAMS = 1 << 25  # the single-thread sample: about 4 s of oracle work per step
+
+
 def oracle_sample_specs(specs):
-    """The bounded CPU sample: the tensors of one transformer layer."""
-    return [i for i, s in enumerate(specs) if s.name.startswith("l0.")]
+    """The bounded CPU sample: the tensors of the first two transformer layers
+    (18 tensors, 404 M params of the 7B layout: at least one tensor per core of
+    a 16-core host); a layout without layers gives its first tensors up to
+    2^26 params."""
+    idx = [i for i, s in enumerate(specs) if s.name.startswith(("l0.", "l1."))]
+    if not idx:
+        total = 0
+        for i, s in enumerate(specs):
+            if idx and total + s.numel > 1 << 26:
+                break
+            idx.append(i)
+            total += s.numel
+    return idx
 
 
-def run_oracle_sample(name: str, steps: int, warmup: int):
-    """Times the CPU oracle, as it stands, on the sample (one thread per
-    tensor; ctypes releases the GIL).  Returns (params/s, ms/step, cores,
-    sample description)."""
+def single_thread_specs(specs, idx):
+    """The single-thread sample: the first tensors of the all-core sample, in
+    layout order, until they hold SINGLE_THREAD_PARAMS params (two 4096^2
+    attention projections of the 7B layout)."""
+    out, total = [], 0
+    for i in idx:
+        if out and total >= SINGLE_THREAD_PARAMS:
+            break
+        out.append(i)
+        total += specs[i].numel
+    return out
+
+
+def run_oracle_sample(name: str, steps: int, warmup: int, single_thread: bool = False):
+    """Times the CPU oracle, as it stands, on a sample of the layout: one host
+    thread per tensor on every available core (ctypes releases the GIL), or
+    one thread in all.  Steps after the first are steady-state (t > 1).
+    Returns (params/s, ms per step of the sample, threads used, sample
+    description)."""
     from concurrent.futures import ThreadPoolExecutor
 
     import numpy as np
@@ -145,6 +175,8 @@ def run_oracle_sample(name: str, steps: int, warmup: int):
     specs = workloads.layout(name)
     cfg = workloads.CFG_ID[name]
     idx = oracle_sample_specs(specs)
+    if single_thread:
+        idx = single_thread_specs(specs, idx)
     sub = [specs[i] for i in idx]
     sig = workloads.tensor_sigmas(specs, cfg)
     sig = [sig[i] for i in idx]
@@ -154,18 +186,18 @@ def run_oracle_sample(name: str, steps: int, warmup: int):
     states = [oracle.TensorState(host.view(host.p, k).numpy(), oracle.E4M3, oracle.E5M2) for k in range(len(sub))]
     grads = [host.view(host.g, k).view(torch.int16).numpy().view(np.uint16) for k in range(len(sub))]
     hp = workloads.HPARAMS
-    cores = min(len(sub), len(os.sched_getaffinity(0)))
+    threads = 1 if single_thread else min(len(sub), len(os.sched_getaffinity(0)))
     n = sum(s.numel for s in sub)
     order = sorted(range(len(sub)), key=lambda k: -sub[k].numel)
 
     def step(t):
         def one(k):
             states[k].step(grads[k], hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], t)
-        with ThreadPoolExecutor(cores) as ex:
+        with ThreadPoolExecutor(threads) as ex:
             list(ex.map(one, order))
 
     t = 0
-    for _ in range(warmup):
+    for _ in range(max(1, warmup)):  # step 1 (with its amax pre-pass) is never timed
         t += 1
         step(t)
     times = []
@@ -175,13 +207,24 @@ def run_oracle_sample(name: str, steps: int, warmup: int):
         step(t)
         times.append(time.perf_counter() - t0)
     ms = 1e3 * sum(times) / len(times)
-    desc = "layer-0 tensors of the %s layout (%d tensors, %d params), steady-state step (t>1), %d host threads" % (
-        name, len(sub), n, cores)
-    return n / (ms / 1e3), ms, cores, desc
+    desc = "%s of the %s layout (%d tensors, %d params), steady-state step (t>1), %d host thread%s" % (
+        "first tensors of layers 0-1" if single_thread else "layers 0-1 (or the first tensors)",
+        name, len(sub), n, threads, "" if threads == 1 else "s, one per tensor")
+    return n / (ms / 1e3), ms, threads, desc
+
+
+def cpu_baseline(name: str, steps: int = 1, warmup: int = 1) -> dict:
+    """The oracle on every available core (the baseline's value) and on one
+    thread, each on its own bounded sample of the layout."""
+    value, ms, threads, desc = run_oracle_sample(name, steps, warmup)
+    v1, ms1, _, desc1 = run_oracle_sample(name, steps, warmup, single_thread=True)
+    return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+            "sample_ms_per_step": ms, "host_cores": len(os.sched_getaffinity(0)),
+            "single_thread": {"value": v1, "unit": UNIT, "cores": 1, "sample": desc1, "sample_ms_per_step": ms1}}
 
 
 def reference_arm(args):
-    from fp8_quantized_adam_b200 import ranks
+    from fp8_quantized_adam_b200 import ranks, workloads
 
     _, rank, _ = ranks.env()
     if rank != 0:
@@ -190,9 +233,15 @@ def reference_arm(args):
 
     oracle.build()
     value, ms, cores, desc = run_oracle_sample(args.workload, args.steps, args.warmup)
+    n_full = workloads.total_params(workloads.layout(args.workload))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup,
+        # the sample's params/s carried to the whole layout; the sample's own
+        # time per step is sample_ms_per_step
+        "ms_per_step": n_full / value * 1e3, "sample_ms_per_step": ms,
+        "ms_per_step_basis": "extrapolated to the full layout (%d params) from the sample's params/s" % n_full,
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(args.workload, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
@@ -215,14 +264,37 @@ def workload_config(name: str, n: int, variant: str = "default") -> dict:
     from fp8_quantized_adam_b200 import workloads
 
     specs = workloads.layout(name)
-    return {"workload": name, "params_per_gpu": workloads.total_params(specs), "tensors": len(specs),
+    n_params = workloads.total_params(specs)
+    gb = BYTES_PER_PARAM * n_params / 1e9
+    l2 = ("inputs larger than L2 (%.1f GB of traffic per step vs 126 MB L2), no flush" % gb if gb > 1.0 else
+          "%.1f MB of traffic per step: partly L2-resident, a latency case, no flush" % (gb * 1e3))
+    return {"workload": name, "params_per_gpu": n_params, "tensors": len(specs),
             "m_fmt": "e4m3", "v_fmt": "e5m2", "grads": "bf16, per-tensor N(0, 10^U(-5,-2)), 0.1% x100",
-            "l2": "inputs larger than L2 (94.3 GB of traffic per step vs 126 MB L2), no flush",
+            "l2": l2,
             "parallelism": "independent shard per GPU x%d" % n, "variant": variant,
             "hparams": {"lr": 3e-4, "beta1": 0.9, "beta2": 0.95, "eps": 1e-8, "weight_decay": 0.1}}
 
 
 # ----------------------------------------------------------------- our arm
+def fail_on_kernel_error(opt, stream, dev, rank: int, where: str) -> None:
+    """Reads the library's device error word (fp8adam_check); if any rank
+    saw an error, rank 0 prints an error line and every rank exits 1.  Every
+    rank takes the same collective (the max over ranks) either way."""
+    from fp8_quantized_adam_b200 import ranks
+
+    err = None
+    try:
+        opt.check(stream)
+    except Exception as ex:  # the library's error, or a CUDA error
+        err = str(ex)
+    if ranks.max_over_ranks(0.0 if err is None else 1.0, dev) == 0.0:
+        return
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "value": None, "unit": UNIT,
+                          "error": "kernel error after the %s: %s" % (where, err or "on another rank")}), flush=True)
+    sys.exit(1)
+
+
 def our_arm(args):
     import torch
 
@@ -283,6 +355,9 @@ def our_arm(args):
     barrier()
     launches = capi.fp8adam_launch_count() - launches0
     clk = clocks.stop()
+    # a staged kernel whose bounded wait ran out leaves its chunk undone and
+    # later CTAs return at once: such a run is faster and wrong, so it ends here
+    fail_on_kernel_error(opt, stream, dev, rank, "timed steps")
     elapsed = t_start.elapsed_time(t_end) / 1e3
     kernel_ms = [a.elapsed_time(b) for a, b in ev]
     elapsed = ranks.max_over_ranks(elapsed, dev)
@@ -312,6 +387,7 @@ def our_arm(args):
                 opt.step_host(host_views, am_host, stream=stream, **step_kw)
             e1.record(stream)
             barrier()
+            fail_on_kernel_error(opt, stream, dev, rank, "end-to-end steps")
             et = ranks.max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
             e2e = {"value": world * n_params * e2e_steps / et, "unit": UNIT,
                    "h2d_bytes_per_step": 2 * n_params,
@@ -344,15 +420,14 @@ def our_arm(args):
                 "frac_of_8TBs_nominal": achieved / 8000.0}
     if args.variant == "sr":
         roofline["note"] = ("stochastic rounding is bound by instruction issue, not DRAM (Philox4x32-10 and the exact "
-                            "SR encoder): profiles/fp8adam_step_ext_tma_kernel_sr_llama2_100m.md")
+                            "SR encoder)")
 
     cpu = None  # the CPU oracle is timed on rank 0 of a 1-GPU run only
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
 
         oracle.build()
-        cv, cms, cores, desc = run_oracle_sample(name, 1, 1)
-        cpu = {"value": cv, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = cpu_baseline(name)
 
     opt.close()
     if rank == 0:
@@ -425,7 +500,8 @@ def ablation_report(args):
                   "flushed_v_mean": sum(out[k]["flushed_v"]) / args.steps,
                   "final_max_abs_dp_vs_fp32": out[k]["max_abs_dp_vs_fp32"][-1], **out[k]}
         del res[k]["ms"]
-    for o in opts.values():
+    for k, o in opts.items():
+        o.check()  # raises if a kernel's bounded wait ran out: no report from a broken run
         o.close()
     print(json.dumps({"report": "format_ablation", "workload": name, "params": n_params, "steps": args.steps,
                       "data": "synthetic", "modes": res}), flush=True)

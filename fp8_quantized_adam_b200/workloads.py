@@ -17,6 +17,10 @@ Fig. 5 moment-format ablation, a Llama2-style 7B model for the headline run):
                   params.
 * ``stress_20k``  20,000 tensors of 4,096 params (grads N(0, 1e-4)) plus 8
                   tensors of 2^28 params (heavy-tailed grads as below).
+* ``pair_2x256m`` two tensors of 2^28 params (heavy-tailed grads): 7.5 GB of
+                  step traffic, 4.3 GB resident -- a launch large enough for
+                  DRAM counters to mean what they mean on the 7B layout, small
+                  enough for a profiler capture.
 
 Heavy-tailed gradients (llama layouts and the 2^28 tensors): per tensor a
 sigma_t = 10^U(-5,-2) drawn once per run; each step g ~ N(0, sigma_t) and a
@@ -33,7 +37,7 @@ import torch
 
 # workload id -> the number used in the seeds
 CFG_ID = {"single_1m": 1, "llama2_100m": 2, "llama2_7b": 3, "ablation_100m": 4,
-          "stress_20k": 5}
+          "stress_20k": 5, "pair_2x256m": 6}
 
 ALIGN_ELEMS = 64  # tensor offsets inside flat buffers: 256 B of fp32, 64 B of codes
 
@@ -71,6 +75,8 @@ def layout(name: str) -> List[TensorSpec]:
     if name == "stress_20k":
         return ([TensorSpec(f"s{i}", 4096, "small") for i in range(20000)]
                 + [TensorSpec(f"b{i}", 1 << 28, "big") for i in range(8)])
+    if name == "pair_2x256m":
+        return [TensorSpec(f"b{i}", 1 << 28, "big") for i in range(2)]
     raise KeyError(name)
 
 
@@ -182,4 +188,4 @@ class FlatModel:
 HPARAMS = dict(lr=3e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1)
 
 STEPS = {"single_1m": 10, "llama2_100m": 100, "llama2_7b": 20, "ablation_100m": 200,
-         "stress_20k": 50}
+         "stress_20k": 50, "pair_2x256m": 20}
