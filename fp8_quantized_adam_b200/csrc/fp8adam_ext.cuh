@@ -69,7 +69,7 @@ __device__ __forceinline__ uint4 sr_words(const ExtArgs& a, int ti, uint32_t t_l
 }
 
 // The same words within one chunk.  A chunk never crosses a multiple of
-// 2^33 elements (its start is a multiple of its power-of-two length), so the
+// 2^33 elements of its tensor (the chunk table is cut there), so the
 // counter's words 1..3 are the same for all its pairs, and so is half of the
 // first round's output: computed once per chunk.
 struct SrChunk {
@@ -98,10 +98,13 @@ __device__ __forceinline__ uint4 sr_words_chunk(const ExtArgs& a, const SrChunk&
 // On the normal grid (2^emin <= |x| < max), the common case, one range test
 // selects the integer path: the spacing is 2^sh fp32 ulps of |x|, the code
 // is |x|'s bits shifted right by sh (rebiased), and the condition is exactly
-// "the top 32 - sh bits of r are below the sh dropped bits".  Below 2^emin
-// the spacing is fixed: y = |x| / spacing is exact, and the threshold is
-// ceil(frac(y) * 2^32).  (Adding 2^emin with round-toward-zero instead, to
-// reuse the integer test, was measured slower.)
+// "the top 32 - sh bits of r are below the sh dropped bits".  It is computed
+// as a carry: adding 2^sh - 1 - (r >> (32 - sh)) to the bits carries into
+// the kept part exactly when (r >> (32 - sh)) < the dropped bits, so the
+// code is one subtract-add and one shift (rebias folded into the constant).
+// Below 2^emin the spacing is fixed: y = |x| / spacing is exact, and the
+// threshold is ceil(frac(y) * 2^32).  (Adding 2^emin with round-toward-zero
+// instead, to reuse the integer test, was measured slower.)
 template <int FMT>
 __device__ __forceinline__ uint32_t enc1_sr(float x, uint32_t r) {
   using T = FmtTraits<FMT>;
@@ -111,7 +114,9 @@ __device__ __forceinline__ uint32_t enc1_sr(float x, uint32_t r) {
   const uint32_t a = u & 0x7FFFFFFFu;
   uint32_t code;
   if (a - kMinNormal < T::kMaxBits - kMinNormal) {  // normal grid, below the max
-    code = ((a - kMinNormal) >> sh) + (1u << T::kMant) + ((r >> (32 - sh)) < (a & ((1u << sh) - 1u)) ? 1u : 0u);
+    // (a - kMinNormal) >> sh + 2^M, plus the carry of the draw (modular: a >= kMinNormal here)
+    constexpr uint32_t kBias = (1u << sh) - 1u + (1u << (T::kMant + sh)) - kMinNormal;
+    code = (a - (r >> (32 - sh)) + kBias) >> sh;
   } else if (a >= T::kMaxBits) {                     // saturate, or NaN
     if (a > 0x7F800000u) return 0x7Fu;
     code = T::kMaxCode;

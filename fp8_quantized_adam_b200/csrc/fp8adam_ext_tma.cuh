@@ -41,7 +41,10 @@ __device__ __forceinline__ uint32_t pack4(uint32_t c0, uint32_t c1, uint32_t c2,
 }
 
 // 4 elements of stage `st` at offset j (global element i, a multiple of 4).
-template <int MF, int VF, bool STATS, bool SR>
+// OPTS: the update-from-stored and bf16-copy options may be on (runtime
+// flags); without them (the lean stochastic-rounding kernel) their code is
+// compiled out.
+template <int MF, int VF, bool STATS, bool SR, bool OPTS>
 __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& st, int j, const TensorDesc& td,
                                              const ExtSeg& sg, const SrChunk& su, int64_t i, float& am, float& av,
                                              uint32_t& flushed, uint32_t& sat) {
@@ -85,7 +88,7 @@ __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& s
   }
   float mu[4] = {mn[0], mn[1], mn[2], mn[3]};
   float vu[4] = {vn[0], vn[1], vn[2], vn[3]};
-  if (a.flags & kExtFromStored) {  // the update reads the stored values
+  if (OPTS && (a.flags & kExtFromStored)) {  // the update reads the stored values
     const float2 qa = dec2_hw<MF>(mq & 0xFFFFu), qb = dec2_hw<MF>(mq >> 16);
     const float2 ra = dec2_hw<VF>(vq & 0xFFFFu), rb = dec2_hw<VF>(vq >> 16);
     mu[0] = __fmul_rn(qa.x, sg.inv_s_m_new);
@@ -111,11 +114,13 @@ __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& s
   st_stream_f4(td.p + i, make_float4(pout[0], pout[1], pout[2], pout[3]));
   __stcs(reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(td.m) + i), mq);
   __stcs(reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(td.v) + i), vq);
-  if (sg.pb)
+  if (OPTS && sg.pb)
     __stcs(reinterpret_cast<uint2*>(sg.pb + i), make_uint2(bf16_pair(pout[0], pout[1]), bf16_pair(pout[2], pout[3])));
 }
 
-template <int MF, int VF, bool STATS, bool SR>
+// SR: stochastic rounding; OPTS as ext_consume4 (the lean SR kernel is
+// launched only when update-from-stored and the bf16 copy are off).
+template <int MF, int VF, bool STATS, bool SR, bool OPTS = true>
 __global__ void __launch_bounds__(kThreads, 4)
 fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   static_assert(MF != kFP32 && VF != kFP32, "the staged path carries 1-byte codes");
@@ -149,7 +154,7 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   SrChunk su{0u, 0u, 0u};
   if constexpr (SR) su = sr_chunk(a, ti, sg.t_lo, e0 >> 1);
   if (!tma_run(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
-        ext_consume4<MF, VF, STATS, SR>(a, st, j, td, sg, su, i, am, av, flushed, sat);
+        ext_consume4<MF, VF, STATS, SR, OPTS>(a, st, j, td, sg, su, i, am, av, flushed, sat);
       }))
     return;
   // the ragged end (under one sub-tile) or an unaligned tensor, element by element
