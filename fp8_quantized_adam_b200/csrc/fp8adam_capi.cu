@@ -165,6 +165,16 @@ ExtFn pick_ext(int mf, int vf, bool stats) {
 }
 using ExtTmaFn = void (*)(const ExtArgs, uint32_t*);
 template <int MF, int VF, bool S, bool SR> ExtTmaFn ext_tma_fn() { return &fp8adam_step_ext_tma_kernel<MF, VF, S, SR>; }
+template <int MF, int VF, bool S> ExtTmaFn ext_tma_lean_fn() { return &fp8adam_step_ext_tma_kernel<MF, VF, S, true, false>; }
+// the lean stochastic-rounding kernel (no update-from-stored, no bf16 copy)
+ExtTmaFn pick_ext_tma_sr_lean(int mf, int vf, bool stats) {  // FP8 formats only
+  static const ExtTmaFn t[2][2][2] = {
+      {{ext_tma_lean_fn<0, 0, false>(), ext_tma_lean_fn<0, 0, true>()},
+       {ext_tma_lean_fn<0, 1, false>(), ext_tma_lean_fn<0, 1, true>()}},
+      {{ext_tma_lean_fn<1, 0, false>(), ext_tma_lean_fn<1, 0, true>()},
+       {ext_tma_lean_fn<1, 1, false>(), ext_tma_lean_fn<1, 1, true>()}}};
+  return t[mf][vf][stats ? 1 : 0];
+}
 ExtTmaFn pick_ext_tma(int mf, int vf, bool stats, bool sr) {  // FP8 formats only
   static const ExtTmaFn t[2][2][2][2] = {
       {{{ext_tma_fn<0, 0, false, false>(), ext_tma_fn<0, 0, false, true>()},
@@ -185,6 +195,11 @@ ExtFn pick_amax_ext(int mf, int vf) {
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Guided chunk lengths (fp8adam_create_ex with chunk_elems 0): see there.
+constexpr int64_t kGuidedRounds = 1;
+constexpr int64_t kGuidedMin = 8192;
+constexpr int64_t kCounterSpan = 1ll << 33;  // a chunk stays within one span of 2^33 elements
 
 // Constants of step t: computed in double, rounded once to fp32.
 StepConsts make_consts(const fp8adam_step_params& p) {
@@ -259,6 +274,7 @@ struct fp8adam_ctx {
   float *scale_m = nullptr, *scale_v = nullptr, *amax_m = nullptr, *amax_v = nullptr;
   TensorDesc* d_tensors = nullptr;
   Chunk* d_chunks = nullptr;
+  ChunkDesc* d_cdesc = nullptr;  // the chunk table with each chunk's tensor buffers (staged step)
   // options of fp8adam_create_ex
   int32_t margin_m = 0, margin_v = 0, hist_len = 0;
   float *hist_m = nullptr, *hist_v = nullptr;
@@ -301,6 +317,7 @@ static void free_ctx(fp8adam_ctx* c) {
   if (!c) return;
   cudaFree(c->d_tensors);
   cudaFree(c->d_chunks);
+  cudaFree(c->d_cdesc);
   cudaFree(c->d_error);
   cudaFree(c->d_bf16);
   cudaFree(c->d_partial);
@@ -394,28 +411,25 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
     cudaGetLastError();
     return FP8ADAM_ERR_CUDA;
   }
-  auto count_chunks = [&](int64_t ce) {
-    int64_t n = 0;
-    for (int32_t i = 0; i < num_tensors; ++i) n += (tensors[i].numel + ce - 1) / ce;
-    return n;
-  };
-  // chunk length: the largest that keeps >= 8 waves of resident CTAs (4 per
-  // SM), so the last partial wave costs little; a list too small for that
-  // gets the shortest chunk (one 4096-element tile), for the most CTAs
-  int64_t chunk = opts->chunk_elems;
-  if (chunk == 0) {
-    const int64_t want = (int64_t)sms * 4 * 8;
-    chunk = kChunk;
-    while (chunk > kTile && count_chunks(chunk) < want) chunk /= 2;
-  }
-  const int64_t total_units = count_chunks(chunk);
-  if (total_units > INT32_MAX / 2) return FP8ADAM_ERR_INVALID_ARG;
-  // the host-side tables (no exception may cross the ABI)
+  // The chunk table: one CTA per chunk, chunks in launch order.  With
+  // chunk_elems set, every chunk has that length (a tensor's last may be
+  // shorter).  Otherwise the lengths are guided by the work still to come:
+  // each chunk takes the remaining elements / (kGuidedRounds x resident
+  // CTAs), rounded down to a whole tile, within [kGuidedMin, kChunk]
+  // (kGuidedRounds 1, 2, 4 and kGuidedMin 4096, 8192 were timed: 1 and 8192
+  // are best on the 100M, 7B and 20K-tensor layouts).  Long
+  // chunks early keep the per-CTA set-up and amax flush rare; the shrinking
+  // chunks at the end of the table leave only a short last wave.  A chunk
+  // never crosses a multiple of 2^33 elements of its tensor (the stochastic-
+  // rounding counter's high word is then constant within a chunk).
+  int64_t total_elems_all = 0;
+  for (int32_t i = 0; i < num_tensors; ++i) total_elems_all += tensors[i].numel;
+  const int64_t slots = (int64_t)sms * 4;  // resident CTAs of the step kernels
   std::vector<TensorDesc> desc;
   std::vector<Chunk> chunks;
   try {
     desc.resize((size_t)num_tensors);
-    chunks.reserve((size_t)total_units);
+    int64_t remaining = total_elems_all;
     for (int32_t i = 0; i < num_tensors; ++i) {
       const fp8adam_tensor& t = tensors[i];
       TensorDesc& d = desc[(size_t)i];
@@ -424,14 +438,30 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
       d.m = t.m;
       d.v = t.v;
       d.numel = t.numel;
-      d.nunits = (int32_t)((t.numel + chunk - 1) / chunk);
       d.aligned = aligned16(t.param) && aligned16(t.grad) && aligned16(t.m) && aligned16(t.v);
-      for (int64_t st = 0; st < t.numel; st += chunk)
-        chunks.push_back(Chunk{i, (int32_t)(t.numel - st < chunk ? t.numel - st : chunk), st});
+      int32_t units = 0;
+      for (int64_t st = 0; st < t.numel;) {
+        int64_t len = opts->chunk_elems;
+        if (len == 0) {
+          len = remaining / (kGuidedRounds * slots) / kTile * kTile;
+          len = len < kGuidedMin ? kGuidedMin : (len > kChunk ? kChunk : len);
+        }
+        const int64_t to_end = t.numel - st;
+        const int64_t to_boundary = (st / kCounterSpan + 1) * kCounterSpan - st;
+        len = std::min(len, std::min(to_end, to_boundary));
+        chunks.push_back(Chunk{i, (int32_t)len, st});
+        st += len;
+        remaining -= len;
+        ++units;
+        if (chunks.size() > (size_t)INT32_MAX / 2) return FP8ADAM_ERR_INVALID_ARG;
+      }
+      d.nunits = units;
     }
   } catch (...) {
     return FP8ADAM_ERR_OOM;
   }
+  const int64_t total_units = (int64_t)chunks.size();
+  const int64_t chunk = opts->chunk_elems;  // 0: guided lengths
 
   fp8adam_ctx* c = new (std::nothrow) fp8adam_ctx();
   if (!c) return FP8ADAM_ERR_OOM;
@@ -452,7 +482,7 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
     int64_t cum = 0, cum_chunks = 0;
     for (int32_t i = 0; i < num_tensors; ++i) {
       cum += tensors[i].numel;
-      cum_chunks += (tensors[i].numel + chunk - 1) / chunk;
+      cum_chunks += desc[(size_t)i].nunits;
       const int g = (int)c->grp_tensor.size();  // groups closed so far + 1
       if (i + 1 == num_tensors || (g < kHostGroups && cum * kHostGroups >= total_elems * g)) {
         c->grp_tensor.push_back(i + 1);
@@ -491,7 +521,26 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
     free_ctx(c);
     return FP8ADAM_ERR_OOM;
   }
-  if (cudaMemcpy(c->d_tensors, desc.data(), T * sizeof(TensorDesc), cudaMemcpyHostToDevice) != cudaSuccess ||
+  std::vector<ChunkDesc> cdesc;
+  try {
+    cdesc.resize(chunks.size());
+  } catch (...) {
+    free_ctx(c);
+    return FP8ADAM_ERR_OOM;
+  }
+  for (size_t k = 0; k < chunks.size(); ++k) {
+    const TensorDesc& d = desc[(size_t)chunks[k].tensor];
+    cdesc[k] = ChunkDesc{d.p, d.g, d.m, d.v, chunks[k].start, d.numel, chunks[k].len, chunks[k].tensor,
+                         d.nunits, d.aligned};
+  }
+  if (cudaMalloc(&c->d_cdesc, (cdesc.empty() ? 1 : cdesc.size()) * sizeof(ChunkDesc)) != cudaSuccess) {
+    cudaGetLastError();
+    free_ctx(c);
+    return FP8ADAM_ERR_OOM;
+  }
+  if ((!cdesc.empty() && cudaMemcpy(c->d_cdesc, cdesc.data(), cdesc.size() * sizeof(ChunkDesc),
+                                    cudaMemcpyHostToDevice) != cudaSuccess) ||
+      cudaMemcpy(c->d_tensors, desc.data(), T * sizeof(TensorDesc), cudaMemcpyHostToDevice) != cudaSuccess ||
       (!chunks.empty() &&
        cudaMemcpy(c->d_chunks, chunks.data(), chunks.size() * sizeof(Chunk), cudaMemcpyHostToDevice) != cudaSuccess) ||
       cudaMemset(c->d_state, 0, 5 * T * sizeof(uint32_t)) != cudaSuccess ||
@@ -519,7 +568,10 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
   if (c->tma && (cudaFuncSetAttribute((const void*)pick_tma(m_fmt, v_fmt, stats_on),
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmemBytes) != cudaSuccess ||
                  cudaFuncSetAttribute((const void*)pick_ext_tma(m_fmt, v_fmt, stats_on, sr_on),
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmemBytes) != cudaSuccess)) {
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmemBytes) != cudaSuccess ||
+                 (sr_on && cudaFuncSetAttribute((const void*)pick_ext_tma_sr_lean(m_fmt, v_fmt, stats_on),
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                kTmaSmemBytes) != cudaSuccess))) {
     cudaGetLastError();
     free_ctx(c);
     return FP8ADAM_ERR_CUDA;
@@ -579,6 +631,7 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
   uint32_t* jit_v = ctx->d_state + 3 * T;
   a.tensors = ctx->d_tensors;
   a.chunks = ctx->d_chunks + c0;
+  a.cdesc = ctx->d_cdesc + c0;
   a.num_tensors = ctx->T;
   a.scale_m = ctx->scale_m;
   a.scale_v = ctx->scale_v;
@@ -663,9 +716,11 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
     a.amax_in_v = reinterpret_cast<const uint32_t*>(ctx->amax_v);
   }
   e.s = a;
-  if (ctx->tma)
-    pick_ext_tma(ctx->m_fmt, ctx->v_fmt, stats, (e.flags & FP8ADAM_FLAG_STOCHASTIC_ROUNDING) != 0)
-        <<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
+  const bool sr = (e.flags & FP8ADAM_FLAG_STOCHASTIC_ROUNDING) != 0;
+  if (ctx->tma && sr && !(e.flags & FP8ADAM_FLAG_UPDATE_FROM_STORED) && !ctx->d_bf16)
+    pick_ext_tma_sr_lean(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
+  else if (ctx->tma)
+    pick_ext_tma(ctx->m_fmt, ctx->v_fmt, stats, sr)<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
   else
     pick_ext(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);

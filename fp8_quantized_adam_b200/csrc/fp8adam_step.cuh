@@ -59,6 +59,22 @@ struct Chunk {
   int64_t start;
 };
 
+// A chunk with what the staged step needs to start it, in one 64-byte
+// record: its tensor's buffers and sizes next to the chunk's range, so a CTA
+// can issue its first copies after a single load.
+struct ChunkDesc {
+  float* p;
+  const uint16_t* g;
+  void* m;
+  void* v;
+  int64_t start;   // first element of the chunk in its tensor
+  int64_t numel;   // the tensor's size
+  int32_t len;     // elements of the chunk
+  int32_t tensor;
+  int32_t nunits;  // chunks of the tensor
+  int32_t aligned; // the tensor's four buffers are 16-byte aligned
+};
+
 struct StepConsts {
   float b1, omb1, b2, omb2, step_size, isbc2, eps, decay;
 };
@@ -79,6 +95,7 @@ struct SchedEntry {
 struct StepArgs {
   const TensorDesc* tensors;     // [T]
   const Chunk* chunks;           // [chunks] tensor and start of each chunk (one per CTA)
+  const ChunkDesc* cdesc;        // [chunks] the same chunks with their tensors' buffers (staged step)
   int32_t num_tensors;
   float* scale_m;            // [T] in: decode scale; out: encode scale of this step
   float* scale_v;

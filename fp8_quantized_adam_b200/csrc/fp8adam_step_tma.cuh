@@ -214,13 +214,26 @@ fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
   __shared__ uint32_t red[4][kThreads / 32];
   __shared__ int abort_flag;
 
-  if (*(volatile const uint32_t*)err) return;  // an earlier CTA timed out: stop at once
-  const Chunk ch = a.chunks[blockIdx.x];
-  const int ti = ch.tensor;
+  // the error word and the chunk's record are loaded together: the first
+  // copies depend on this one load only
+  const uint32_t err_word = *(volatile const uint32_t*)err;
+  const ChunkDesc cd = a.cdesc[blockIdx.x];
+  if (err_word) return;  // an earlier CTA timed out: stop at once
+  const int ti = cd.tensor;
   FP8ADAM_BOUNDS(ti >= 0 && ti < a.num_tensors);
-  const TensorDesc td = a.tensors[ti];
+  TensorDesc td;
+  td.p = cd.p;
+  td.g = cd.g;
+  td.m = cd.m;
+  td.v = cd.v;
+  td.numel = cd.numel;
+  td.nunits = cd.nunits;
+  td.aligned = cd.aligned;
+#ifdef FP8ADAM_DEBUG
+  td.numel = a.tensors[ti].numel;  // the debug build checks against the tensor table (set by a debug hook)
+#endif
   if (a.cur && !a.cur->valid) return;  // a scheduled step past the end of its schedule
-  const int64_t e0 = ch.start, e1 = ch.start + ch.len;
+  const int64_t e0 = cd.start, e1 = cd.start + cd.len;
   FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
   // whole sub-tiles go through the staged pipeline (aligned tensors only);
   // the first copies are issued before the per-tensor loads below

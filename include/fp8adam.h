@@ -205,10 +205,14 @@ typedef struct {
   uint16_t* const* param_bf16; /* host array [num_tensors] of device bf16 buffers
                                   [numel] receiving the updated params rounded to
                                   nearest even (entries may be NULL), or NULL */
-  int32_t chunk_elems;       /* elements per CTA: 0 = chosen from the list's size
-                                (the largest power of two in [4096, 131072]
-                                giving at least 8 waves of CTAs, else 4096);
-                                otherwise a multiple of 4096 in [4096, 131072].
+  int32_t chunk_elems;       /* elements per CTA: 0 = guided by the work left
+                                (each chunk, in launch order, takes the
+                                elements still to come / resident CTAs,
+                                rounded down to a multiple of 4096 within
+                                [8192, 131072]); otherwise a multiple of 4096
+                                in [4096, 131072].  A tensor's last chunk, and
+                                one that would cross a multiple of 2^33
+                                elements of its tensor, is cut shorter.
                                 Results do not depend on it. */
 } fp8adam_options;
 
