@@ -157,7 +157,7 @@ def test_current_scaling_every_step():
 
 def test_edge_sizes_and_misaligned_views():
     """Sizes around the 16-element vector, the 4096-element tile and the
-    chunk lengths the library picks (16384 .. 131072), an empty tensor, and
+    chunk lengths the library picks (8192 .. 131072), an empty tensor, and
     tensors whose buffers are offset by one element (element-by-element
     path)."""
     sizes = [0, 1, 15, 16, 17, 4095, 4096, 4097, 16383, 16385, 65535, 65536, 65537, 131071, 131073,
