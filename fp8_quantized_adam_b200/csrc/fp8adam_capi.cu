@@ -614,8 +614,10 @@ static float host_multiplier(const fp8adam_step_params& p) {
 // `cur` (a scheduled step): the kernels take the constants and per-step
 // options from that device entry instead of `p`; whether the pre-passes run
 // is then decided per schedule (grad norm) or per context (JIT amax).
+// `pdl`: launch the staged default step with programmatic dependent launch
+// (the steps of fp8adam_step / fp8adam_step_ex, back to back on a stream).
 static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t st, int32_t c0, int32_t c1,
-                          bool first, const SchedEntry* cur = nullptr) {
+                          bool first, const SchedEntry* cur = nullptr, bool pdl = false) {
   if (c1 <= c0) return FP8ADAM_OK;  // only empty tensors
   const bool prepass = cur ? ctx->sched_prepass : needs_prepass(p);
   const bool ext = ctx->ext || prepass || (!cur && p.loss_scale != 1.0f);
@@ -661,7 +663,25 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
       a.amax_in_m = reinterpret_cast<const uint32_t*>(ctx->amax_m);
       a.amax_in_v = reinterpret_cast<const uint32_t*>(ctx->amax_v);
     }
-    if (ctx->tma)
+    if (ctx->tma && pdl) {
+      // the kernel may start while the previous kernel on the stream finishes
+      // (it waits for that kernel's writes with griddepcontrol.wait)
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = grid;
+      cfg.blockDim = block;
+      cfg.dynamicSmemBytes = kTmaSmemBytes;
+      cfg.stream = st;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      uint32_t* err = ctx->d_error;
+      if (cudaLaunchKernelEx(&cfg, pick_tma(ctx->m_fmt, ctx->v_fmt, stats), a, err) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8ADAM_ERR_CUDA;
+      }
+    } else if (ctx->tma)
       pick_tma(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, kTmaSmemBytes, st>>>(a, ctx->d_error);
     else
       pick_step(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(a);
@@ -732,7 +752,7 @@ static int run_step(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return FP8ADAM_ERR_CUDA;
   if (dev != ctx->device) return FP8ADAM_ERR_WRONG_DEVICE;
-  return run_step_range(ctx, p, st, 0, ctx->total_units, true);
+  return run_step_range(ctx, p, st, 0, ctx->total_units, true, nullptr, true);
 }
 
 extern "C" int fp8adam_step(fp8adam_ctx* ctx, float lr, float beta1, float beta2, float eps,

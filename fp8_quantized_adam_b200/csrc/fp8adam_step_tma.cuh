@@ -214,10 +214,18 @@ fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
   __shared__ uint32_t red[4][kThreads / 32];
   __shared__ int abort_flag;
 
-  // the error word and the chunk's record are loaded together: the first
-  // copies depend on this one load only
-  const uint32_t err_word = *(volatile const uint32_t*)err;
+  // The chunk's record is static (written at create), so it is read before
+  // the previous kernel in the stream has finished.  With programmatic
+  // dependent launch (the step launched back to back with the previous one),
+  // this grid starts while that kernel's last CTAs still run: every CTA lets
+  // the next step's grid start once all of this grid's CTAs have started,
+  // and waits for the previous grid's writes before it reads anything they
+  // may touch (params, moments, scales, amax, counters, the error word).
+  // Launched without it, both instructions return at once.
   const ChunkDesc cd = a.cdesc[blockIdx.x];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const uint32_t err_word = *(volatile const uint32_t*)err;
   if (err_word) return;  // an earlier CTA timed out: stop at once
   const int ti = cd.tensor;
   FP8ADAM_BOUNDS(ti >= 0 && ti < a.num_tensors);

@@ -121,8 +121,11 @@ int fp8adam_create(const fp8adam_tensor* tensors, int32_t num_tensors,
  * on `cuda_stream` (a cudaStream_t; NULL = legacy default stream).  Requires
  * 0 <= beta1, beta2 < 1, eps >= 0, finite lr and weight_decay, step >= 1;
  * otherwise INVALID_ARG with nothing queued.  At step 1 (or every step with
- * FP8ADAM_FLAG_JIT_EVERY_STEP) an amax pre-pass runs first.  Returns CUDA if
- * a launch fails. */
+ * FP8ADAM_FLAG_JIT_EVERY_STEP) an amax pre-pass runs first.  The staged step
+ * kernel is launched with programmatic dependent launch: it may start while
+ * the previous kernel on the stream finishes, and reads nothing that kernel
+ * can write before that kernel has completed (results are unchanged).
+ * Returns CUDA if a launch fails. */
 int fp8adam_step(fp8adam_ctx* ctx, float lr, float beta1, float beta2,
                  float eps, float weight_decay, int64_t step,
                  void* cuda_stream);
