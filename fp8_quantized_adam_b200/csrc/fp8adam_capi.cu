@@ -425,6 +425,9 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
   int64_t total_elems_all = 0;
   for (int32_t i = 0; i < num_tensors; ++i) total_elems_all += tensors[i].numel;
   const int64_t slots = (int64_t)sms * 4;  // resident CTAs of the step kernels
+  // a list that does not fill one wave of kGuidedMin chunks (a latency case)
+  // gets one-tile chunks, for the most CTAs
+  const int64_t guided_min = total_elems_all < slots * kGuidedMin ? kTile : kGuidedMin;
   std::vector<TensorDesc> desc;
   std::vector<Chunk> chunks;
   try {
@@ -444,7 +447,7 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
         int64_t len = opts->chunk_elems;
         if (len == 0) {
           len = remaining / (kGuidedRounds * slots) / kTile * kTile;
-          len = len < kGuidedMin ? kGuidedMin : (len > kChunk ? kChunk : len);
+          len = len < guided_min ? guided_min : (len > kChunk ? kChunk : len);
         }
         const int64_t to_end = t.numel - st;
         const int64_t to_boundary = (st / kCounterSpan + 1) * kCounterSpan - st;

@@ -10,8 +10,8 @@
 // Design for B200: the step is a pure HBM stream (read p 4 B, g 2 B, m 1 B,
 // v 1 B; write p 4 B, m 1 B, v 1 B per element).  One launch covers a whole
 // parameter list through a chunk table: CTA b handles chunk b, a run of
-// elements of one tensor (the chunk length is chosen per parameter list so
-// the grid has many waves; up to kChunk), 4 CTAs of 256 threads resident per
+// elements of one tensor (lengths guided by the work still to come: long
+// chunks first, short ones last; up to kChunk), 4 CTAs of 256 threads resident per
 // SM (64 registers).  Each thread moves 16 elements per iteration with 16-byte
 // loads and stores (4 x p, 2 x g, 1 x m, 1 x v), streaming cache hints, all
 // fp32 arithmetic as single IEEE operations (no FMA contraction), hardware

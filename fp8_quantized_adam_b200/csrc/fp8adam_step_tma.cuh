@@ -12,7 +12,7 @@
 // on registers.  4 CTAs of 256 threads per SM (62-64 registers, 48 KB of
 // shared memory each).  A chunk's first copies are issued before its
 // per-tensor loads and scale arithmetic, which then overlap the fill.
-// Measured on the 7B-shaped layout: 14.15 ms per step against 14.85 ms for
+// Measured on the 7B-shaped layout: 14.12 ms per step against 14.85 ms for
 // per-thread vector loads and 14.1 ms for a probe with the same copies and no
 // arithmetic; a warp-specialised form (separate producer warp, empty/full
 // barriers) and 1024-element sub-tiles were slower.

@@ -212,7 +212,9 @@ typedef struct {
                                 (each chunk, in launch order, takes the
                                 elements still to come / resident CTAs,
                                 rounded down to a multiple of 4096 within
-                                [8192, 131072]); otherwise a multiple of 4096
+                                [8192, 131072], or [4096, 131072] for a list
+                                too small to fill one wave of 8192-element
+                                chunks); otherwise a multiple of 4096
                                 in [4096, 131072].  A tensor's last chunk, and
                                 one that would cross a multiple of 2^33
                                 elements of its tensor, is cut shorter.

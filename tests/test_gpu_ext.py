@@ -13,6 +13,7 @@ import pytest
 import torch
 
 import oracle
+import pins
 from fp8_quantized_adam_b200 import FP8AdamW, capi, workloads
 from gpu_harness import HP, bf16_host_bits
 
@@ -253,3 +254,64 @@ def test_options_on_the_llama2_100m_layout():
     for _ in range(3):
         r.step()
     r.compare()
+
+
+@pytest.mark.slow
+def test_stochastic_rounding_counter_beyond_2_pow_33():
+    """One tensor of 2^33 + 2*4096 + 5 elements, stochastic rounding on,
+    inputs periodic in 4096 elements, step 1 from the zero state.  Element j's
+    random words are Philox4x32-10 of counter (j/2 low, j/2 high, tensor,
+    step): past element 2^33 the counter's high word changes, and the chunk
+    table is cut there.  The codes of sampled elements on both sides of 2^33
+    and at the end must equal the oracle's SR encoder fed with the oracle's
+    Philox bits for those very indices; the params (which do not depend on the
+    rounding) equal the oracle's step on one period, bit for bit."""
+    period = 4096
+    n = (1 << 33) + 2 * period + 5
+    seed = 0x5EED0FF1CE
+    dev = torch.device("cuda:0")
+    base = workloads.custom_layout([period])
+    pp = torch.zeros(period)
+    workloads.init_params_into(base, [pp], 53)
+    gg = torch.zeros(period, dtype=torch.bfloat16)
+    workloads.grads_into(base, [gg], 53, 1, workloads.tensor_sigmas(base, 53))
+    reps = (n + period - 1) // period
+    p = pp.to(dev).repeat(reps)[:n]
+    g = gg.to(dev).repeat(reps)[:n]
+    m = torch.zeros(n, dtype=torch.uint8, device=dev)
+    v = torch.zeros(n, dtype=torch.uint8, device=dev)
+    opt = FP8AdamW([p], [g], m=[m], v=[v], stochastic_rounding=True, seed=seed)
+    opt.step()
+    opt.check()
+    # the oracle on one period: the scales (from the step-1 amax, equal for
+    # the periodic tensor) and the params
+    ref = oracle.TensorState(pp.numpy(), oracle.E4M3, oracle.E5M2)
+    gbits = bf16_host_bits(gg)
+    ref.step_ex(gbits, HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], 1,
+                oracle.FLAG_STOCHASTIC, seed=seed, tensor_index=0)
+    assert float(opt.scale_m[0]) == float(ref.scale_m[0]) and float(opt.scale_v[0]) == float(ref.scale_v[0])
+    assert float(opt.amax_m[0]) == float(ref.amax_m[0]) and float(opt.amax_v[0]) == float(ref.amax_v[0])
+    # step 1 from zero moments: m = 0 + (1 - b1) g and v = 0 + (1 - b2) g^2, one
+    # fp32 rounding each, as the oracle's op order has them
+    c = oracle.step_constants(HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], 1)
+    omb1, omb2 = np.float32(c[1]), np.float32(c[3])
+    gf = pins.bf16_bits_to_f32(gbits)
+    s_m, s_v = np.float32(ref.scale_m[0]), np.float32(ref.scale_v[0])
+    two33 = 1 << 33
+    starts = [two33 - 3 * period - 64, two33 - 64, two33 + period - 64, n - 200]  # all inside [0, n - 192]
+    assert all(0 <= st and st + 192 <= n for st in starts)
+    for st in starts:
+        k = 192
+        got_m = m[st:st + k].cpu().numpy()
+        got_v = v[st:st + k].cpu().numpy()
+        got_p = p[st:st + k].cpu().numpy()
+        for o in range(k):
+            j = st + o
+            gj = gf[j % period]
+            xm = np.float32(np.float32(omb1 * gj) * s_m)
+            xv = np.float32(np.float32(omb2 * np.float32(gj * gj)) * s_v)
+            em = oracle.encode_sr(oracle.E4M3, float(xm), oracle.sr_bits(seed, 0, 1, j, 0))
+            ev = oracle.encode_sr(oracle.E5M2, float(xv), oracle.sr_bits(seed, 0, 1, j, 1))
+            assert got_m[o] == em and got_v[o] == ev, (j, got_m[o], em, got_v[o], ev)
+        assert (got_p.view(np.uint32) == ref.p[(np.arange(st, st + k) % period)].view(np.uint32)).all()
+    opt.close()
