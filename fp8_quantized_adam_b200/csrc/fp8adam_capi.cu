@@ -166,7 +166,8 @@ ExtFn pick_ext(int mf, int vf, bool stats) {
 using ExtTmaFn = void (*)(const ExtArgs, uint32_t*);
 template <int MF, int VF, bool S, bool SR> ExtTmaFn ext_tma_fn() { return &fp8adam_step_ext_tma_kernel<MF, VF, S, SR>; }
 template <int MF, int VF, bool S> ExtTmaFn ext_tma_lean_fn() { return &fp8adam_step_ext_tma_kernel<MF, VF, S, true, false>; }
-// the lean stochastic-rounding kernel (no update-from-stored, no bf16 copy)
+// the lean stochastic-rounding kernel (no update-from-stored, no bf16 copy,
+// gradient multiplier 1)
 ExtTmaFn pick_ext_tma_sr_lean(int mf, int vf, bool stats) {  // FP8 formats only
   static const ExtTmaFn t[2][2][2] = {
       {{ext_tma_lean_fn<0, 0, false>(), ext_tma_lean_fn<0, 0, true>()},
@@ -740,7 +741,8 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
   }
   e.s = a;
   const bool sr = (e.flags & FP8ADAM_FLAG_STOCHASTIC_ROUNDING) != 0;
-  if (ctx->tma && sr && !(e.flags & FP8ADAM_FLAG_UPDATE_FROM_STORED) && !ctx->d_bf16)
+  if (ctx->tma && sr && !(e.flags & FP8ADAM_FLAG_UPDATE_FROM_STORED) && !ctx->d_bf16 && e.grad_mult == nullptr &&
+      e.gm_const == 1.0f)
     pick_ext_tma_sr_lean(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
   else if (ctx->tma)
     pick_ext_tma(ctx->m_fmt, ctx->v_fmt, stats, sr)<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);

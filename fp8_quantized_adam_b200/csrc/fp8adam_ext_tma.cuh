@@ -42,8 +42,8 @@ __device__ __forceinline__ uint32_t pack4(uint32_t c0, uint32_t c1, uint32_t c2,
 
 // 4 elements of stage `st` at offset j (global element i, a multiple of 4).
 // OPTS: the update-from-stored and bf16-copy options may be on (runtime
-// flags); without them (the lean stochastic-rounding kernel) their code is
-// compiled out.
+// flags) and the gradient multiplier may differ from 1; without them (the
+// lean stochastic-rounding kernel) their code is compiled out.
 template <int MF, int VF, bool STATS, bool SR, bool OPTS>
 __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& st, int j, const TensorDesc& td,
                                              const ExtSeg& sg, const SrChunk& su, int64_t i, float& am, float& av,
@@ -60,8 +60,11 @@ __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& s
                        __fmul_rn(mb.y, sg.inv_s_m)};
   const float vo[4] = {__fmul_rn(va.x, sg.inv_s_v), __fmul_rn(va.y, sg.inv_s_v), __fmul_rn(vb.x, sg.inv_s_v),
                        __fmul_rn(vb.y, sg.inv_s_v)};
-  const float g[4] = {__fmul_rn(bf16_lo(gq.x), sg.gm), __fmul_rn(bf16_hi(gq.x), sg.gm),
-                      __fmul_rn(bf16_lo(gq.y), sg.gm), __fmul_rn(bf16_hi(gq.y), sg.gm)};
+  // the lean instance runs only with the multiplier 1 (no loss scale, no clipping)
+  const float g[4] = {OPTS ? __fmul_rn(bf16_lo(gq.x), sg.gm) : bf16_lo(gq.x),
+                      OPTS ? __fmul_rn(bf16_hi(gq.x), sg.gm) : bf16_hi(gq.x),
+                      OPTS ? __fmul_rn(bf16_lo(gq.y), sg.gm) : bf16_lo(gq.y),
+                      OPTS ? __fmul_rn(bf16_hi(gq.y), sg.gm) : bf16_hi(gq.y)};
   const float p4[4] = {pin.x, pin.y, pin.z, pin.w};
   float mn[4], vn[4], ym[4], yv[4];
 #pragma unroll
@@ -119,7 +122,8 @@ __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& s
 }
 
 // SR: stochastic rounding; OPTS as ext_consume4 (the lean SR kernel is
-// launched only when update-from-stored and the bf16 copy are off).
+// launched only when update-from-stored and the bf16 copy are off and the
+// gradient multiplier is 1).
 template <int MF, int VF, bool STATS, bool SR, bool OPTS = true>
 __global__ void __launch_bounds__(kThreads, 4)
 fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {

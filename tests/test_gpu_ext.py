@@ -123,6 +123,17 @@ def test_stochastic_rounding(fmts, tma):
         r.compare()
 
 
+def test_stochastic_rounding_with_a_loss_scale():
+    """Stochastic rounding with a loss scale and no clipping: the multiplier
+    1/loss_scale is a kernel argument, so the staged kernel that keeps the
+    multiply runs (the lean one assumes multiplier 1); codes, params, scales
+    and amax equal the oracle's bit for bit."""
+    r = ExtRun(54, stochastic_rounding=True, seed=0xABCDEF)
+    for ls in (4.0, 1000.0, 1.0, 65536.0):
+        r.step(loss_scale=ls)
+        r.compare()
+
+
 @pytest.mark.parametrize("tma", [True, False], ids=["staged", "vector"])
 def test_bf16_param_copy(tma):
     r = ExtRun(44, bf16=True, tma=tma)
@@ -245,7 +256,7 @@ def test_options_through_host_step():
 def test_options_on_the_llama2_100m_layout():
     """Stochastic rounding, a 16-step history, margins and the bf16 copy on
     the 110-tensor Llama2-100M layout in the launch configuration the bench
-    times (16K-element chunks, staged kernel); the embedding, the first and
+    times (guided chunk table, staged kernel); the embedding, the first and
     last layer's matrices and a norm gain against the oracle, bit for bit."""
     specs = workloads.layout("llama2_100m")
     subset = [0, 1, 5, len(specs) - 2, len(specs) - 1]
