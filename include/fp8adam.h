@@ -369,8 +369,7 @@ uint64_t fp8adam_launch_count(void);
  * - A NaN moment gives the canonical NaN amax (bits 0x7FFFFFFF), as the
  *   regular step does.
  * - The first call on a device looks up the scratch array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   (cudaGetSymbolAddress) with that device current.
  * - Each call copies the tensor table from host memory into the scratch
  *   (the copy waits for work already queued on cuda_stream) and clears the
  *   accumulators, so no state carries over between calls.
