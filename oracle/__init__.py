@@ -25,6 +25,7 @@ E4M3, E5M2, FP32 = 0, 1, 2
 FLAG_JIT_EVERY_STEP = 2
 FLAG_UPDATE_FROM_STORED = 4
 FLAG_STOCHASTIC = 8
+FLAG_SR_DRAW16 = 32  # with FLAG_STOCHASTIC: 16-bit draws
 
 
 class StepOpts(ctypes.Structure):
@@ -89,6 +90,18 @@ def lib() -> ctypes.CDLL:
         L.ref_encode_sr.argtypes = [c_int, c_f, c_u32]
         L.ref_encode_sr_array.restype = None
         L.ref_encode_sr_array.argtypes = [c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, c_i64]
+        L.ref_rev16.restype = c_u32
+        L.ref_rev16.argtypes = [c_u32]
+        L.ref_sr16_draw.restype = c_u32
+        L.ref_sr16_draw.argtypes = [c_u32, c_int]
+        L.ref_encode_sr16.restype = c_u32
+        L.ref_encode_sr16.argtypes = [c_int, c_f, c_u32]
+        L.ref_encode_sr16_array.restype = None
+        L.ref_encode_sr16_array.argtypes = [c_int, vp, vp, vp, c_i64]
+        L.ref_encode_sr16_words.restype = None
+        L.ref_encode_sr16_words.argtypes = [c_int, vp, vp, vp, c_i64]
+        L.ref_sr16_bits.restype = c_u32
+        L.ref_sr16_bits.argtypes = [ctypes.c_uint64, ctypes.c_int32, c_i64, c_i64, c_int]
         L.ref_f32_to_bf16.restype = ctypes.c_uint16
         L.ref_f32_to_bf16.argtypes = [c_f]
         L.ref_f32_to_bf16_array.restype = None
@@ -151,6 +164,43 @@ def sr_bits(seed: int, tensor: int, t: int, j: int, which: int) -> int:
 
 def encode_sr(fmt: int, x: float, r: int) -> int:
     return int(lib().ref_encode_sr(fmt, x, r))
+
+
+def rev16(x: int) -> int:
+    return int(lib().ref_rev16(x))
+
+
+def sr16_draw(w: int, k: int) -> int:
+    """The 16-bit draw of code k (0..3) among the four codes word w serves."""
+    return int(lib().ref_sr16_draw(w, k))
+
+
+def encode_sr16(fmt: int, x: float, r16: int) -> int:
+    return int(lib().ref_encode_sr16(fmt, x, r16))
+
+
+def encode_sr16_array(fmt: int, x, r16) -> np.ndarray:
+    """Codes of x[j] stochastically rounded with the 16-bit draws r16[j]."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    r = np.ascontiguousarray(r16, dtype=np.uint32)
+    assert x.shape == r.shape
+    out = np.empty(x.size, np.uint8)
+    lib().ref_encode_sr16_array(fmt, _ptr(x), _ptr(r), _ptr(out), x.size)
+    return out
+
+
+def encode_sr16_words(fmt: int, x, w) -> np.ndarray:
+    """Codes of x[j] with the draw of code j % 4 of word w[j // 4]."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    w = np.ascontiguousarray(w, dtype=np.uint32)
+    assert w.size * 4 >= x.size
+    out = np.empty(x.size, np.uint8)
+    lib().ref_encode_sr16_words(fmt, _ptr(x), _ptr(w), _ptr(out), x.size)
+    return out
+
+
+def sr16_bits(seed: int, tensor: int, t: int, j: int, which: int) -> int:
+    return int(lib().ref_sr16_bits(seed, tensor, t, j, which))
 
 
 def encode_sr_array(fmt: int, x, r) -> np.ndarray:

@@ -236,3 +236,15 @@ def sr_cases(fmt: int, seed: int):
     rs.append(rng.integers(0, 1 << 32, spec.size, dtype=np.uint64).astype(np.uint32))
     up.append(np.full(spec.size, -1, np.int8))
     return np.concatenate(xs).astype(np.float32), np.concatenate(rs), np.concatenate(up)
+
+
+def sr16_threshold(fmt: int, x: np.ndarray):
+    """For finite |x| below the format's max: (lo, hi, F) with lo <= |x| < hi
+    neighbours on the torch float8 grid and F = floor((|x| - lo) / (hi - lo) *
+    2^16); a 16-bit draw r rounds up iff F + r >= 2^16.  float64 is exact as
+    in sr_threshold."""
+    grid = finite_grid(fmt)
+    a = np.abs(np.asarray(x, np.float64))
+    k = np.searchsorted(grid, a, side="right") - 1
+    lo, hi = grid[k], grid[k + 1]
+    return lo, hi, np.floor((a - lo) / (hi - lo) * 65536.0)
