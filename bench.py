@@ -262,7 +262,7 @@ def kernel_name(args) -> str:
         k = "fp8adam_step_kernel<E4M3,E5M2>" if args.no_tma else "fp8adam_step_tma_kernel<E4M3,E5M2>"
         return k + (" + amax pre-pass" if args.variant == "jit" else "")
     base = ("fp8adam_step_ext_kernel<E4M3,E5M2>" if args.no_tma else
-            "fp8adam_step_ext_tma_kernel<E4M3,E5M2,SR=%d>" % (args.variant == "sr"))
+            "fp8adam_step_ext_tma_kernel<E4M3,E5M2,SRK=%d>" % {"sr": 1, "sr16": 2}.get(args.variant, 0))
     return base + (" + grad-norm pre-pass" if args.variant == "clip" else "")
 
 
@@ -328,6 +328,8 @@ def our_arm(args):
     opt_kw, step_kw = {}, {}
     if args.variant == "sr":
         opt_kw = dict(stochastic_rounding=True, seed=1234)
+    elif args.variant == "sr16":
+        opt_kw = dict(stochastic_rounding=True, seed=1234, sr_draw_bits=16)
     elif args.variant == "history":
         opt_kw = dict(amax_history_len=16)
     elif args.variant == "jit":
@@ -441,8 +443,11 @@ def our_arm(args):
                                      "note": "a second pass of the same steps, each between its own CUDA events"},
                 "frac_of_8TBs_nominal": achieved / 8000.0}
     if args.variant == "sr":
-        roofline["note"] = ("stochastic rounding is bound by instruction issue, not DRAM (Philox4x32-10 and the exact "
-                            "SR encoder)")
+        roofline["note"] = ("stochastic rounding with 32-bit draws is bound by instruction issue, not DRAM "
+                            "(Philox4x32-10 for every two elements and the integer SR encoder)")
+    elif args.variant == "sr16":
+        roofline["note"] = ("stochastic rounding with 16-bit draws: one Philox4x32-10 call per eight elements, "
+                            "four codes per hardware stochastic-rounding conversion")
 
     cpu = None  # the CPU oracle is timed on rank 0 of a 1-GPU run only
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -539,7 +544,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--chunk-elems", type=int, default=0, help="elements per CTA (0: chosen by the library)")
     ap.add_argument("--no-tma", action="store_true", help="per-thread vector loads instead of TMA staging")
-    ap.add_argument("--variant", choices=["default", "sr", "history", "clip", "jit"], default="default",
+    ap.add_argument("--variant", choices=["default", "sr", "sr16", "history", "clip", "jit"], default="default",
                     help="step options: stochastic rounding, amax history 16, fused loss-scale/clip/skip, "
                          "current scaling (amax pre-pass every step)")
     ap.add_argument("--no-e2e", action="store_true")

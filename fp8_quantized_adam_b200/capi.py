@@ -31,6 +31,7 @@ FLAG_STATS = 1
 FLAG_JIT_EVERY_STEP = 2
 FLAG_UPDATE_FROM_STORED = 4
 FLAG_STOCHASTIC_ROUNDING = 8
+FLAG_SR_DRAW16 = 32  # with FLAG_STOCHASTIC_ROUNDING: 16-bit draws, hardware conversion
 FLAG_NO_TMA = 16
 
 
@@ -112,6 +113,8 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
                                     vp, vp]
     L.fp8adam_encode_sr.restype = ctypes.c_int
     L.fp8adam_encode_sr.argtypes = [i32, vp, vp, vp, i64, vp]
+    L.fp8adam_encode_sr16.restype = ctypes.c_int
+    L.fp8adam_encode_sr16.argtypes = [i32, vp, vp, vp, i64, vp]
     L.fp8adam_launch_count.restype = ctypes.c_uint64
     L.fp8adam_launch_count.argtypes = []
     L.fp8adam_create_ex.restype = ctypes.c_int
@@ -234,6 +237,10 @@ def fp8adam_encode_sr(fmt: int, x: int, r: int, out: int, n: int, cuda_stream: i
     _check("fp8adam_encode_sr", lib().fp8adam_encode_sr(fmt, x, r, out, n, cuda_stream))
 
 
+def fp8adam_encode_sr16(fmt: int, x: int, w: int, out: int, n: int, cuda_stream: int) -> None:
+    _check("fp8adam_encode_sr16", lib().fp8adam_encode_sr16(fmt, x, w, out, n, cuda_stream))
+
+
 def fp8adam_decode(fmt: int, codes: int, out: int, n: int, impl: int, cuda_stream: int) -> None:
     _check("fp8adam_decode", lib().fp8adam_decode(fmt, codes, out, n, impl, cuda_stream))
 
@@ -255,6 +262,7 @@ def fp8adam_step_noalloc(tensors, num_tensors: int, scale_m: int, scale_v: int, 
 EXPORTED = ["fp8adam_create", "fp8adam_step", "fp8adam_get_stats", "fp8adam_reset_stats",
             "fp8adam_destroy", "fp8adam_strerror", "fp8adam_encode", "fp8adam_encode_bits_range",
             "fp8adam_decode", "fp8adam_launch_count", "fp8adam_step_noalloc", "fp8adam_create_ex",
-            "fp8adam_step_ex", "fp8adam_get_grad_info", "fp8adam_check", "fp8adam_encode_sr", "fp8adam_step_host",
+            "fp8adam_step_ex", "fp8adam_get_grad_info", "fp8adam_check", "fp8adam_encode_sr", "fp8adam_encode_sr16",
+            "fp8adam_step_host",
             "fp8adam_debug_inject_wait", "fp8adam_debug_set_numel", "fp8adam_set_schedule",
             "fp8adam_step_scheduled", "fp8adam_get_schedule_step"]

@@ -108,6 +108,27 @@ __global__ void encode_sr_kernel(const float* __restrict__ x, const uint32_t* __
     out[i] = (uint8_t)enc1_sr<FMT>(x[i], r[i]);
 }
 
+// four codes per word: out[4q + k] = code k of x[4q .. 4q+3] rounded with
+// word w[q] (inputs past n are 0 and their codes are not written)
+template <int FMT>
+__global__ void encode_sr16_kernel(const float* __restrict__ x, const uint32_t* __restrict__ w,
+                                   uint8_t* __restrict__ out, int64_t n) {
+  const int64_t nw = (n + 3) >> 2;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < nw; q += stride) {
+    const int64_t i = q << 2;
+    const float x0 = x[i];
+    const float x1 = i + 1 < n ? x[i + 1] : 0.0f;
+    const float x2 = i + 2 < n ? x[i + 2] : 0.0f;
+    const float x3 = i + 3 < n ? x[i + 3] : 0.0f;
+    const uint32_t d = cvt_rs4<FMT>(x0, x1, x2, x3, w[q]);
+    out[i] = (uint8_t)d;
+    if (i + 1 < n) out[i + 1] = (uint8_t)(d >> 8);
+    if (i + 2 < n) out[i + 2] = (uint8_t)(d >> 16);
+    if (i + 3 < n) out[i + 3] = (uint8_t)(d >> 24);
+  }
+}
+
 int grid_for(int64_t n, int per_thread) {
   const int64_t want = (n + (int64_t)256 * per_thread - 1) / ((int64_t)256 * per_thread);
   const int64_t cap = 148 * 16;
@@ -164,29 +185,31 @@ ExtFn pick_ext(int mf, int vf, bool stats) {
   return t[mf][vf][stats ? 1 : 0];
 }
 using ExtTmaFn = void (*)(const ExtArgs, uint32_t*);
-template <int MF, int VF, bool S, bool SR> ExtTmaFn ext_tma_fn() { return &fp8adam_step_ext_tma_kernel<MF, VF, S, SR>; }
-template <int MF, int VF, bool S> ExtTmaFn ext_tma_lean_fn() { return &fp8adam_step_ext_tma_kernel<MF, VF, S, true, false>; }
-// the lean stochastic-rounding kernel (no update-from-stored, no bf16 copy,
-// gradient multiplier 1)
-ExtTmaFn pick_ext_tma_sr_lean(int mf, int vf, bool stats) {  // FP8 formats only
-  static const ExtTmaFn t[2][2][2] = {
-      {{ext_tma_lean_fn<0, 0, false>(), ext_tma_lean_fn<0, 0, true>()},
-       {ext_tma_lean_fn<0, 1, false>(), ext_tma_lean_fn<0, 1, true>()}},
-      {{ext_tma_lean_fn<1, 0, false>(), ext_tma_lean_fn<1, 0, true>()},
-       {ext_tma_lean_fn<1, 1, false>(), ext_tma_lean_fn<1, 1, true>()}}};
-  return t[mf][vf][stats ? 1 : 0];
+// srk: the rounding kind (0 nearest, 1 stochastic with 32-bit draws, 2 with
+// 16-bit draws)
+template <int MF, int VF, bool S, int K> ExtTmaFn ext_tma_fn() { return &fp8adam_step_ext_tma_kernel<MF, VF, S, K>; }
+template <int MF, int VF, bool S, int K> ExtTmaFn ext_tma_lean_fn() {
+  return &fp8adam_step_ext_tma_kernel<MF, VF, S, K, false>;
 }
-ExtTmaFn pick_ext_tma(int mf, int vf, bool stats, bool sr) {  // FP8 formats only
-  static const ExtTmaFn t[2][2][2][2] = {
-      {{{ext_tma_fn<0, 0, false, false>(), ext_tma_fn<0, 0, false, true>()},
-        {ext_tma_fn<0, 0, true, false>(), ext_tma_fn<0, 0, true, true>()}},
-       {{ext_tma_fn<0, 1, false, false>(), ext_tma_fn<0, 1, false, true>()},
-        {ext_tma_fn<0, 1, true, false>(), ext_tma_fn<0, 1, true, true>()}}},
-      {{{ext_tma_fn<1, 0, false, false>(), ext_tma_fn<1, 0, false, true>()},
-        {ext_tma_fn<1, 0, true, false>(), ext_tma_fn<1, 0, true, true>()}},
-       {{ext_tma_fn<1, 1, false, false>(), ext_tma_fn<1, 1, false, true>()},
-        {ext_tma_fn<1, 1, true, false>(), ext_tma_fn<1, 1, true, true>()}}}};
-  return t[mf][vf][stats ? 1 : 0][sr ? 1 : 0];
+template <int MF, int VF, bool S> struct ExtTmaRow {
+  ExtTmaFn k[3] = {ext_tma_fn<MF, VF, S, 0>(), ext_tma_fn<MF, VF, S, 1>(), ext_tma_fn<MF, VF, S, 2>()};
+  ExtTmaFn lean[2] = {ext_tma_lean_fn<MF, VF, S, 1>(), ext_tma_lean_fn<MF, VF, S, 2>()};
+};
+template <bool S> const ExtTmaFn* ext_tma_row(int mf, int vf, bool lean) {  // FP8 formats only
+  static const ExtTmaRow<0, 0, S> r00;
+  static const ExtTmaRow<0, 1, S> r01;
+  static const ExtTmaRow<1, 0, S> r10;
+  static const ExtTmaRow<1, 1, S> r11;
+  if (mf == 0) return vf == 0 ? (lean ? r00.lean : r00.k) : (lean ? r01.lean : r01.k);
+  return vf == 0 ? (lean ? r10.lean : r10.k) : (lean ? r11.lean : r11.k);
+}
+// the lean stochastic-rounding kernels (no update-from-stored, no bf16 copy,
+// gradient multiplier 1); srk 1 or 2
+ExtTmaFn pick_ext_tma_sr_lean(int mf, int vf, bool stats, int srk) {
+  return (stats ? ext_tma_row<true>(mf, vf, true) : ext_tma_row<false>(mf, vf, true))[srk - 1];
+}
+ExtTmaFn pick_ext_tma(int mf, int vf, bool stats, int srk) {
+  return (stats ? ext_tma_row<true>(mf, vf, false) : ext_tma_row<false>(mf, vf, false))[srk];
 }
 ExtFn pick_amax_ext(int mf, int vf) {
   static const ExtFn t[3][3] = {{aext_fn<0, 0>(), aext_fn<0, 1>(), aext_fn<0, 2>()},
@@ -196,6 +219,16 @@ ExtFn pick_amax_ext(int mf, int vf) {
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static_assert(FP8ADAM_FLAG_UPDATE_FROM_STORED == kExtFromStored && FP8ADAM_FLAG_STOCHASTIC_ROUNDING == kExtStochastic &&
+                  FP8ADAM_FLAG_SR_DRAW16 == kExtSrDraw16,
+              "the step passes these flag bits to the kernels unchanged");
+
+// the rounding kind of a flag set (0 nearest, 1 SR with 32-bit draws, 2 SR with 16-bit draws)
+int sr_kind_of(uint32_t flags) {
+  if (!(flags & FP8ADAM_FLAG_STOCHASTIC_ROUNDING)) return 0;
+  return (flags & FP8ADAM_FLAG_SR_DRAW16) ? 2 : 1;
+}
 
 // Guided chunk lengths (fp8adam_create_ex with chunk_elems 0): see there.
 constexpr int64_t kGuidedRounds = 1;
@@ -369,7 +402,9 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
     return FP8ADAM_ERR_INVALID_ARG;
   if (m_fmt < 0 || m_fmt > 2 || v_fmt < 0 || v_fmt > 2) return FP8ADAM_ERR_UNSUPPORTED_FMT;
   if (flags & ~(FP8ADAM_FLAG_STATS | FP8ADAM_FLAG_JIT_EVERY_STEP | FP8ADAM_FLAG_UPDATE_FROM_STORED |
-                FP8ADAM_FLAG_STOCHASTIC_ROUNDING | FP8ADAM_FLAG_NO_TMA))
+                FP8ADAM_FLAG_STOCHASTIC_ROUNDING | FP8ADAM_FLAG_NO_TMA | FP8ADAM_FLAG_SR_DRAW16))
+    return FP8ADAM_ERR_INVALID_ARG;
+  if ((flags & FP8ADAM_FLAG_SR_DRAW16) && !(flags & FP8ADAM_FLAG_STOCHASTIC_ROUNDING))
     return FP8ADAM_ERR_INVALID_ARG;
   if (opts->chunk_elems < 0 || opts->chunk_elems > kChunk || opts->chunk_elems % kTile != 0)
     return FP8ADAM_ERR_INVALID_ARG;
@@ -568,14 +603,14 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
   }
   c->tma = m_fmt != FP8ADAM_FP32 && v_fmt != FP8ADAM_FP32 && !(flags & FP8ADAM_FLAG_NO_TMA);
   const bool stats_on = (flags & FP8ADAM_FLAG_STATS) != 0;
-  const bool sr_on = (flags & FP8ADAM_FLAG_STOCHASTIC_ROUNDING) != 0;
+  const int srk = sr_kind_of(flags);
   if (c->tma && (cudaFuncSetAttribute((const void*)pick_tma(m_fmt, v_fmt, stats_on),
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmemBytes) != cudaSuccess ||
-                 cudaFuncSetAttribute((const void*)pick_ext_tma(m_fmt, v_fmt, stats_on, sr_on),
+                 cudaFuncSetAttribute((const void*)pick_ext_tma(m_fmt, v_fmt, stats_on, srk),
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmemBytes) != cudaSuccess ||
-                 (sr_on && cudaFuncSetAttribute((const void*)pick_ext_tma_sr_lean(m_fmt, v_fmt, stats_on),
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                kTmaSmemBytes) != cudaSuccess))) {
+                 (srk && cudaFuncSetAttribute((const void*)pick_ext_tma_sr_lean(m_fmt, v_fmt, stats_on, srk),
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              kTmaSmemBytes) != cudaSuccess))) {
     cudaGetLastError();
     free_ctx(c);
     return FP8ADAM_ERR_CUDA;
@@ -694,7 +729,7 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
   }
 
   ExtArgs e;
-  e.flags = ctx->flags & (FP8ADAM_FLAG_UPDATE_FROM_STORED | FP8ADAM_FLAG_STOCHASTIC_ROUNDING);
+  e.flags = ctx->flags & (FP8ADAM_FLAG_UPDATE_FROM_STORED | FP8ADAM_FLAG_STOCHASTIC_ROUNDING | FP8ADAM_FLAG_SR_DRAW16);
   e.margin_m = ctx->margin_m;
   e.margin_v = ctx->margin_v;
   e.use_hist = (ctx->hist_len > 1 && !jit) ? 1 : 0;
@@ -740,12 +775,12 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
     a.amax_in_v = reinterpret_cast<const uint32_t*>(ctx->amax_v);
   }
   e.s = a;
-  const bool sr = (e.flags & FP8ADAM_FLAG_STOCHASTIC_ROUNDING) != 0;
-  if (ctx->tma && sr && !(e.flags & FP8ADAM_FLAG_UPDATE_FROM_STORED) && !ctx->d_bf16 && e.grad_mult == nullptr &&
+  const int srk = sr_kind_of(e.flags);
+  if (ctx->tma && srk && !(e.flags & FP8ADAM_FLAG_UPDATE_FROM_STORED) && !ctx->d_bf16 && e.grad_mult == nullptr &&
       e.gm_const == 1.0f)
-    pick_ext_tma_sr_lean(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
+    pick_ext_tma_sr_lean(ctx->m_fmt, ctx->v_fmt, stats, srk)<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
   else if (ctx->tma)
-    pick_ext_tma(ctx->m_fmt, ctx->v_fmt, stats, sr)<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
+    pick_ext_tma(ctx->m_fmt, ctx->v_fmt, stats, srk)<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
   else
     pick_ext(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -1107,6 +1142,18 @@ extern "C" int fp8adam_encode_sr(int32_t fmt, const float* x, const uint32_t* r,
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   if (fmt == 0) encode_sr_kernel<0><<<grid_for(n, 1), 256, 0, st>>>(x, r, out, n);
   else encode_sr_kernel<1><<<grid_for(n, 1), 256, 0, st>>>(x, r, out, n);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return last_error();
+}
+
+extern "C" int fp8adam_encode_sr16(int32_t fmt, const float* x, const uint32_t* w, uint8_t* out, int64_t n,
+                                   void* cuda_stream) {
+  if (fmt < 0 || fmt > 1) return FP8ADAM_ERR_UNSUPPORTED_FMT;
+  if (n < 0 || (n > 0 && (!x || !w || !out))) return FP8ADAM_ERR_INVALID_ARG;
+  if (n == 0) return FP8ADAM_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (fmt == 0) encode_sr16_kernel<0><<<grid_for(n, 4), 256, 0, st>>>(x, w, out, n);
+  else encode_sr16_kernel<1><<<grid_for(n, 4), 256, 0, st>>>(x, w, out, n);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return last_error();
 }

@@ -11,7 +11,9 @@
 //     case, sub-section "一个数值例子");
 //   - stochastic rounding of the codes ("随机舍入" in "应对FP8训练稳定性挑战的
 //     策略"), with random bits from Philox4x32-10 (Salmon, Moraes, Dror, Shaw,
-//     "Parallel random numbers: as easy as 1, 2, 3", SC 2011);
+//     "Parallel random numbers: as easy as 1, 2, 3", SC 2011): 32-bit draws
+//     with the integer encoder below, or 16-bit draws rounded by the
+//     hardware's stochastic-rounding conversion (four codes per instruction);
 //   - a fused gradient multiplier (loss-scale removal and global-norm
 //     clipping: "梯度缩放", "梯度裁剪" and the clip_grad_norm_ example) and
 //     skip-on-non-finite, fed by a deterministic grad-norm pre-pass;
@@ -29,6 +31,7 @@ namespace fp8adam {
 enum ExtFlags : uint32_t {
   kExtFromStored = 4u,  // the update reads dec(code)/scale
   kExtStochastic = 8u,  // stochastic rounding of the codes
+  kExtSrDraw16 = 32u,   // with kExtStochastic: 16-bit draws, rounded by the hardware conversion
 };
 
 struct ExtArgs {
@@ -131,6 +134,32 @@ __device__ __forceinline__ uint32_t enc1_sr(float x, uint32_t r) {
   return ((u >> 24) & 0x80u) | code;
 }
 
+// ------------------------------------------------------------ SR with 16-bit draws
+// cvt.rs.satfinite.{e4m3x4,e5m2x4}.f32 (sm_100a): four values to four codes
+// in one instruction, each rounded stochastically with 16 random bits: up iff
+// floor((|x|-lo)/(hi-lo) * 2^16) + r >= 2^16, saturating to the largest
+// finite code, NaN -> 0x7F.  Byte k of the result is the code of xk; x0
+// takes the word's low half as r, x1 the low half with its bits in reverse
+// order, x2 the high half, x3 the high half reversed.
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt_rs4(float x0, float x1, float x2, float x3, uint32_t w) {
+  uint32_t d;
+  if constexpr (FMT == kE4M3)
+    asm("cvt.rs.satfinite.e4m3x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=r"(d) : "f"(x3), "f"(x2), "f"(x1), "f"(x0), "r"(w));
+  else
+    asm("cvt.rs.satfinite.e5m2x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=r"(d) : "f"(x3), "f"(x2), "f"(x1), "f"(x0), "r"(w));
+  return d;
+}
+
+// One value as code `lane` (0..3) of word w (the other three inputs are 0,
+// which every draw leaves at code 0).
+template <int FMT>
+__device__ __forceinline__ uint32_t enc1_sr16(float x, uint32_t w, int lane) {
+  const uint32_t d = cvt_rs4<FMT>(lane == 0 ? x : 0.0f, lane == 1 ? x : 0.0f, lane == 2 ? x : 0.0f,
+                                  lane == 3 ? x : 0.0f, w);
+  return (d >> (8 * lane)) & 0xFFu;
+}
+
 // ------------------------------------------------------------ scale with margin
 template <int FMT>
 __device__ __forceinline__ float pow2scale_margin(float amax, float s_prev, int margin) {
@@ -154,24 +183,37 @@ __device__ __forceinline__ float pow2scale_margin(float amax, float s_prev, int 
 // ------------------------------------------------------------ encode/store
 // Rounding of the codes: fixed at compile time (the staged kernels, one
 // instantiation each) or read from ExtArgs::flags (the per-thread-load kernel).
-enum SrMode : int { kRoundNearest = 0, kRoundStochastic = 1, kRoundByFlag = 2 };
+enum SrMode : int { kRoundNearest = 0, kRoundStochastic = 1, kRoundByFlag = 2, kRoundStochastic16 = 3 };
 
+// 0: round to nearest; 1: SR with 32-bit draws; 2: SR with 16-bit draws
 template <int SRM>
-__device__ __forceinline__ bool use_sr(const ExtArgs& a) {
-  if constexpr (SRM == kRoundByFlag) return (a.flags & kExtStochastic) != 0;
-  else return SRM == kRoundStochastic;
+__device__ __forceinline__ int sr_kind(const ExtArgs& a) {
+  if constexpr (SRM == kRoundByFlag)
+    return (a.flags & kExtStochastic) ? ((a.flags & kExtSrDraw16) ? 2 : 1) : 0;
+  else if constexpr (SRM == kRoundStochastic) return 1;
+  else if constexpr (SRM == kRoundStochastic16) return 2;
+  else return 0;
 }
 
+// The random words of elements i .. i+3 (i a multiple of 4) for m and v.
+// 32-bit draws: one word per code, from the call of pair i/2 and i/2 + 1
+// (.x/.y of a call: m/v of its even element, .z/.w: of its odd element).
+// 16-bit draws: one word per four codes, from the call of i/8 (.x/.y: m/v of
+// elements 8q .. 8q+3, .z/.w: of 8q+4 .. 8q+7).
+
 // Encodes one moment value (x * s) and returns the value the update reads.
+// r: the element's 32-bit draw, or (16-bit draws) the word of its four codes,
+// of which it is code `lane`.
 template <int FMT, bool STATS, bool IS_V, int SRM>
-__device__ __forceinline__ float ext_q(const ExtArgs& a, float x, float s, float inv_s, uint32_t r, uint32_t& code,
-                                       uint32_t& flushed, uint32_t& sat) {
+__device__ __forceinline__ float ext_q(const ExtArgs& a, float x, float s, float inv_s, uint32_t r, int lane,
+                                       uint32_t& code, uint32_t& flushed, uint32_t& sat) {
   if constexpr (FMT == kFP32) {
     code = 0;
     return x;
   } else {
     const float y = __fmul_rn(x, s);
-    code = use_sr<SRM>(a) ? enc1_sr<FMT>(y, r) : enc1_hw<FMT>(y);
+    const int k = sr_kind<SRM>(a);
+    code = k == 1 ? enc1_sr<FMT>(y, r) : (k == 2 ? enc1_sr16<FMT>(y, r, lane) : enc1_hw<FMT>(y));
     if constexpr (STATS) {
       sat += fabsf(y) > FmtTraits<FMT>::kMax ? 1u : 0u;
       if constexpr (IS_V) flushed += (x > 0.0f && (code & 0x7Fu) == 0u) ? 1u : 0u;
@@ -196,10 +238,15 @@ __device__ __forceinline__ void ext_element(const ExtArgs& a, const TensorDesc& 
   FP8ADAM_BOUNDS(i >= 0 && i < td.numel);
   const StepConsts& c = sg.c;
   uint32_t rm = 0, rv = 0;
-  if (use_sr<SRM>(a)) {
+  const int srk = sr_kind<SRM>(a);
+  if (srk == 1) {
     const uint4 r = sr_words(a, sg.ti, sg.t_lo, i >> 1);
     rm = (i & 1) ? r.z : r.x;
     rv = (i & 1) ? r.w : r.y;
+  } else if (srk == 2) {
+    const uint4 r = sr_words(a, sg.ti, sg.t_lo, i >> 3);
+    rm = ((i >> 2) & 1) ? r.z : r.x;
+    rv = ((i >> 2) & 1) ? r.w : r.y;
   }
   const float g = __fmul_rn(__uint_as_float((uint32_t)td.g[i] << 16), sg.gm);
   float mn, vn;
@@ -207,8 +254,9 @@ __device__ __forceinline__ void ext_element(const ExtArgs& a, const TensorDesc& 
   am = fmax_nan(am, fabsf(mn));
   av = fmax_nan(av, fabsf(vn));
   uint32_t qm, qv;
-  const float mu = ext_q<MF, STATS, false, SRM>(a, mn, sg.s_m_new, sg.inv_s_m_new, rm, qm, flushed, sat);
-  const float vu = ext_q<VF, STATS, true, SRM>(a, vn, sg.s_v_new, sg.inv_s_v_new, rv, qv, flushed, sat);
+  const int lane = (int)(i & 3);
+  const float mu = ext_q<MF, STATS, false, SRM>(a, mn, sg.s_m_new, sg.inv_s_m_new, rm, lane, qm, flushed, sat);
+  const float vu = ext_q<VF, STATS, true, SRM>(a, vn, sg.s_v_new, sg.inv_s_v_new, rv, lane, qv, flushed, sat);
   if constexpr (MF == kFP32) static_cast<float*>(td.m)[i] = mn; else static_cast<uint8_t*>(td.m)[i] = (uint8_t)qm;
   if constexpr (VF == kFP32) static_cast<float*>(td.v)[i] = vn; else static_cast<uint8_t*>(td.v)[i] = (uint8_t)qv;
   const float pn = update(c, td.p[i], mu, vu);
@@ -240,21 +288,27 @@ __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& 
     tv.decode4(k, sg.inv_s_v, vo);
     const float g[4] = {__fmul_rn(bf16_lo(gw[2 * k]), sg.gm), __fmul_rn(bf16_hi(gw[2 * k]), sg.gm),
                         __fmul_rn(bf16_lo(gw[2 * k + 1]), sg.gm), __fmul_rn(bf16_hi(gw[2 * k + 1]), sg.gm)};
-    uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
-    if (use_sr<SRM>(a)) {
-      r0 = sr_words(a, sg.ti, sg.t_lo, (i + 4 * k) >> 1);
-      r1 = sr_words(a, sg.ti, sg.t_lo, ((i + 4 * k) >> 1) + 1);
+    uint32_t rmj[4] = {0, 0, 0, 0}, rvj[4] = {0, 0, 0, 0};
+    const int srk = sr_kind<SRM>(a);
+    if (srk == 1) {
+      const uint4 r0 = sr_words(a, sg.ti, sg.t_lo, (i + 4 * k) >> 1);
+      const uint4 r1 = sr_words(a, sg.ti, sg.t_lo, ((i + 4 * k) >> 1) + 1);
+      rmj[0] = r0.x; rmj[1] = r0.z; rmj[2] = r1.x; rmj[3] = r1.z;
+      rvj[0] = r0.y; rvj[1] = r0.w; rvj[2] = r1.y; rvj[3] = r1.w;
+    } else if (srk == 2) {  // i + 4k is a multiple of 4: one word for the four m codes, one for the v codes
+      const uint4 r = sr_words(a, sg.ti, sg.t_lo, (i + 4 * k) >> 3);
+      const bool second = (((i + 4 * k) >> 2) & 1) != 0;
+      rmj[0] = rmj[1] = rmj[2] = rmj[3] = second ? r.z : r.x;
+      rvj[0] = rvj[1] = rvj[2] = rvj[3] = second ? r.w : r.y;
     }
-    const uint32_t rmj[4] = {r0.x, r0.z, r1.x, r1.z};
-    const uint32_t rvj[4] = {r0.y, r0.w, r1.y, r1.w};
     uint32_t qm[4], qv[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       moments(c, g[j], mo[j], vo[j], mn[j], vn[j]);
       am = fmax_nan(am, fabsf(mn[j]));
       av = fmax_nan(av, fabsf(vn[j]));
-      mu[j] = ext_q<MF, STATS, false, SRM>(a, mn[j], sg.s_m_new, sg.inv_s_m_new, rmj[j], qm[j], flushed, sat);
-      vu[j] = ext_q<VF, STATS, true, SRM>(a, vn[j], sg.s_v_new, sg.inv_s_v_new, rvj[j], qv[j], flushed, sat);
+      mu[j] = ext_q<MF, STATS, false, SRM>(a, mn[j], sg.s_m_new, sg.inv_s_m_new, rmj[j], j, qm[j], flushed, sat);
+      vu[j] = ext_q<VF, STATS, true, SRM>(a, vn[j], sg.s_v_new, sg.inv_s_v_new, rvj[j], j, qv[j], flushed, sat);
     }
     float pk[4] = {pv[k].x, pv[k].y, pv[k].z, pv[k].w};
 #pragma unroll

@@ -9,9 +9,11 @@
 //     grad-norm pre-pass, or a host constant 1/loss_scale without one), one
 //     multiply;
 //   - the encode scales from the amax history and the margin (per chunk);
-//   - stochastic rounding (a compile-time switch: Philox4x32-10 words for two
-//     elements per call, and the integer SR encoder), or round-to-nearest
-//     with the hardware conversion;
+//   - the rounding (a compile-time kind): round-to-nearest with the hardware
+//     conversion; stochastic rounding with 32-bit draws (Philox4x32-10 words
+//     for two elements per call, and the integer SR encoder); or stochastic
+//     rounding with 16-bit draws (one call per eight elements, four codes per
+//     hardware stochastic-rounding conversion);
 //   - the update from the stored moments (a uniform branch: decode the new
 //     codes again);
 //   - the bf16 copy of the new params (a uniform branch: one 8-byte store
@@ -41,13 +43,16 @@ __device__ __forceinline__ uint32_t pack4(uint32_t c0, uint32_t c1, uint32_t c2,
 }
 
 // 4 elements of stage `st` at offset j (global element i, a multiple of 4).
-// OPTS: the update-from-stored and bf16-copy options may be on (runtime
-// flags) and the gradient multiplier may differ from 1; without them (the
-// lean stochastic-rounding kernel) their code is compiled out.
-template <int MF, int VF, bool STATS, bool SR, bool OPTS>
+// SRK: 0 round to nearest, 1 stochastic with 32-bit draws (computed here
+// from su), 2 stochastic with 16-bit draws (the words wm, wv of the four m
+// and the four v codes, from the caller).  OPTS: the update-from-stored and
+// bf16-copy options may be on (runtime flags) and the gradient multiplier may
+// differ from 1; without them (the lean stochastic-rounding kernels) their
+// code is compiled out.
+template <int MF, int VF, bool STATS, int SRK, bool OPTS>
 __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& st, int j, const TensorDesc& td,
-                                             const ExtSeg& sg, const SrChunk& su, int64_t i, float& am, float& av,
-                                             uint32_t& flushed, uint32_t& sat) {
+                                             const ExtSeg& sg, const SrChunk& su, uint32_t wm, uint32_t wv,
+                                             int64_t i, float& am, float& av, uint32_t& flushed, uint32_t& sat) {
   FP8ADAM_BOUNDS(i >= 0 && i + 4 <= td.numel);
   const StepConsts& c = sg.c;
   const float4 pin = *reinterpret_cast<const float4*>(&st.p[j]);
@@ -76,7 +81,7 @@ __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& s
     yv[e] = __fmul_rn(vn[e], sg.s_v_new);
   }
   uint32_t mq, vq;
-  if constexpr (SR) {
+  if constexpr (SRK == 1) {
     // words of elements (i, i+1) and (i+2, i+3): .x/.y = m/v of the even
     // element, .z/.w = m/v of the odd one
     const uint4 r0 = sr_words_chunk(a, su, (uint32_t)(i >> 1));
@@ -85,6 +90,9 @@ __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& s
                enc1_sr<MF>(ym[3], r1.z));
     vq = pack4(enc1_sr<VF>(yv[0], r0.y), enc1_sr<VF>(yv[1], r0.w), enc1_sr<VF>(yv[2], r1.y),
                enc1_sr<VF>(yv[3], r1.w));
+  } else if constexpr (SRK == 2) {
+    mq = cvt_rs4<MF>(ym[0], ym[1], ym[2], ym[3], wm);
+    vq = cvt_rs4<VF>(yv[0], yv[1], yv[2], yv[3], wv);
   } else {
     mq = enc2_hw<MF>(ym[0], ym[1]) | (enc2_hw<MF>(ym[2], ym[3]) << 16);
     vq = enc2_hw<VF>(yv[0], yv[1]) | (enc2_hw<VF>(yv[2], yv[3]) << 16);
@@ -121,13 +129,15 @@ __device__ __forceinline__ void ext_consume4(const ExtArgs& a, const TmaStage& s
     __stcs(reinterpret_cast<uint2*>(sg.pb + i), make_uint2(bf16_pair(pout[0], pout[1]), bf16_pair(pout[2], pout[3])));
 }
 
-// SR: stochastic rounding; OPTS as ext_consume4 (the lean SR kernel is
-// launched only when update-from-stored and the bf16 copy are off and the
+// SRK: the rounding kind of ext_consume4; OPTS as there (the lean SR kernels
+// are launched only when update-from-stored and the bf16 copy are off and the
 // gradient multiplier is 1).
-template <int MF, int VF, bool STATS, bool SR, bool OPTS = true>
+template <int MF, int VF, bool STATS, int SRK, bool OPTS = true>
 __global__ void __launch_bounds__(kThreads, 4)
 fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   static_assert(MF != kFP32 && VF != kFP32, "the staged path carries 1-byte codes");
+  static_assert(SRK != 2 || (kSub == 8 * kThreads && kTile % 8 == 0 && kSub % 8 == 0),
+                "16-bit draws: two groups of four per thread and stage, chunks starting at multiples of 8");
   extern __shared__ __align__(128) unsigned char tma_smem[];
   TmaStage* stage = reinterpret_cast<TmaStage*>(tma_smem);
   __shared__ __align__(8) uint64_t full[kStages];
@@ -156,14 +166,39 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   uint32_t flushed = 0, sat = 0;
 
   SrChunk su{0u, 0u, 0u};
-  if constexpr (SR) su = sr_chunk(a, ti, sg.t_lo, e0 >> 1);
+  if constexpr (SRK == 1) su = sr_chunk(a, ti, sg.t_lo, e0 >> 1);
+  if constexpr (SRK == 2) su = sr_chunk(a, ti, sg.t_lo, e0 >> 3);
+  uint32_t w1m = 0, w1v = 0;  // 16-bit draws: the words of this thread's second group of the stage
   if (!tma_run(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
-        ext_consume4<MF, VF, STATS, SR, OPTS>(a, st, j, td, sg, su, i, am, av, flushed, sat);
+        uint32_t wm = 0, wv = 0;
+        if constexpr (SRK == 2) {
+          if (j < 4 * kThreads) {
+            // The stage's first group of thread t is elements i .. i+3 (i = 8q
+            // for even t, 8q + 4 for odd t), its second i + 1024 .. i + 1027.
+            // One Philox call per thread and stage: even t takes the call of
+            // its first group's eight elements (its own four and those of
+            // t + 1), odd t that of its second group's (those of t - 1 and its
+            // own); each passes the neighbour the two words it needs.
+            const bool odd = (threadIdx.x & 1u) != 0;
+            const uint4 w = sr_words_chunk(a, su, (uint32_t)((odd ? i + 4 * kThreads : i) >> 3));
+            const uint32_t g0 = __shfl_xor_sync(0xFFFFFFFFu, odd ? w.x : w.z, 1);
+            const uint32_t g1 = __shfl_xor_sync(0xFFFFFFFFu, odd ? w.y : w.w, 1);
+            wm = odd ? g0 : w.x;
+            wv = odd ? g1 : w.y;
+            w1m = odd ? w.z : g0;
+            w1v = odd ? w.w : g1;
+          } else {
+            wm = w1m;
+            wv = w1v;
+          }
+        }
+        ext_consume4<MF, VF, STATS, SRK, OPTS>(a, st, j, td, sg, su, wm, wv, i, am, av, flushed, sat);
       }))
     return;
   // the ragged end (under one sub-tile) or an unaligned tensor, element by element
+  constexpr int kElemRound = SRK == 1 ? kRoundStochastic : (SRK == 2 ? kRoundStochastic16 : kRoundNearest);
   for (int64_t i = e0 + (int64_t)nsub * kSub + threadIdx.x; i < e1; i += kThreads)
-    ext_element<MF, VF, STATS, SR ? kRoundStochastic : kRoundNearest>(a, td, sg, i, am, av, flushed, sat);
+    ext_element<MF, VF, STATS, kElemRound>(a, td, sg, i, am, av, flushed, sat);
   ext_flush<STATS>(a, ti, td.nunits, sg, am, av, flushed, sat, red);
 }
 

@@ -33,7 +33,9 @@ class FP8AdamW:
     Options (fp8adam_create_ex): ``margin_m``/``margin_v`` (scale margin),
     ``amax_history_len`` (scale from the max of the last N amax; the ring is
     allocated here and checkpointed), ``update_from_stored`` (the update reads
-    the requantised moments), ``stochastic_rounding`` with ``seed``, and
+    the requantised moments), ``stochastic_rounding`` with ``seed`` and
+    ``sr_draw_bits`` (32: the integer encoder with 32-bit draws; 16: 16-bit
+    draws rounded by the hardware's stochastic-rounding conversion), and
     ``param_bf16`` (bf16 tensors receiving the updated params).  Per step:
     ``step(loss_scale=, max_norm=, skip_nonfinite=)`` (fp8adam_step_ex).
     """
@@ -46,11 +48,13 @@ class FP8AdamW:
                  amax_v: Optional[torch.Tensor] = None, stats: bool = False,
                  jit_every_step: bool = False, margin_m: int = 0, margin_v: int = 0,
                  amax_history_len: int = 0, update_from_stored: bool = False,
-                 stochastic_rounding: bool = False, seed: int = 0,
+                 stochastic_rounding: bool = False, seed: int = 0, sr_draw_bits: int = 32,
                  param_bf16: Optional[List[torch.Tensor]] = None, chunk_elems: int = 0,
                  tma: bool = True):
         if len(params) == 0 or len(params) != len(grads):
             raise ValueError("need matching, non-empty param and grad lists")
+        if sr_draw_bits not in (16, 32):
+            raise ValueError("sr_draw_bits is 32 or 16")
         self.params, self.grads = list(params), list(grads)
         dev = self.params[0].device
         if dev.type != "cuda":
@@ -103,6 +107,7 @@ class FP8AdamW:
         flags = ((capi.FLAG_STATS if stats else 0) | (capi.FLAG_JIT_EVERY_STEP if jit_every_step else 0)
                  | (capi.FLAG_UPDATE_FROM_STORED if update_from_stored else 0)
                  | (capi.FLAG_STOCHASTIC_ROUNDING if stochastic_rounding else 0)
+                 | (capi.FLAG_SR_DRAW16 if sr_draw_bits == 16 else 0)
                  | (0 if tma else capi.FLAG_NO_TMA))
         self.amax_history_len = int(amax_history_len)
         self.hist_m = self.hist_v = None

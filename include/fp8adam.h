@@ -181,6 +181,15 @@ const char* fp8adam_strerror(int code);
  * update from stored moments. */
 #define FP8ADAM_FLAG_UPDATE_FROM_STORED 4u   /* the update reads dec(code)/scale */
 #define FP8ADAM_FLAG_STOCHASTIC_ROUNDING 8u  /* codes rounded stochastically */
+/* With FP8ADAM_FLAG_STOCHASTIC_ROUNDING (INVALID_ARG without it): 16-bit
+ * draws instead of 32-bit ones, rounded by the B200's stochastic-rounding
+ * conversion (cvt.rs, four codes per instruction, one Philox4x32-10 call per
+ * eight elements).  Code of element j: up iff floor((|x|-lo)/(hi-lo) * 2^16)
+ * + r >= 2^16, r the draw of code j % 4 of word 2*((j/4) % 2) + (0 for m, 1
+ * for v) of the call with counter (j/8 low, j/8 high, tensor, step), draws as
+ * fp8adam_encode_sr16 takes them.  The probability of rounding up is the
+ * exact one rounded down to a multiple of 2^-16. */
+#define FP8ADAM_FLAG_SR_DRAW16 32u
 
 typedef struct {
   float* scale_m;            /* as fp8adam_create: device fp32 [num_tensors] */
@@ -336,6 +345,20 @@ int fp8adam_encode_bits_range(int32_t fmt, uint32_t first, int64_t n,
  * "FP8训练的稳定性挑战…". */
 int fp8adam_encode_sr(int32_t fmt, const float* x, const uint32_t* r,
                       uint8_t* out, int64_t n, void* cuda_stream);
+
+/* Stochastic rounding with 16-bit draws and caller-given words: out[j] = the
+ * code of x[j], rounded up to hi iff floor((|x[j]|-lo)/(hi-lo) * 2^16) + r >=
+ * 2^16, with r the draw of code j % 4 from word w[j / 4]: code 0 takes the
+ * word's low 16 bits, code 1 the low 16 bits in reverse bit order, code 2 the
+ * high 16 bits, code 3 the high 16 bits reversed; saturating to the largest
+ * finite code; NaN -> 0x7F.  The encoder of FP8ADAM_FLAG_SR_DRAW16, one
+ * hardware conversion per word.  x, out: device arrays of n elements; w:
+ * device array of (n + 3) / 4 words.  Returns INVALID_ARG for n < 0 or a NULL
+ * pointer with n > 0, UNSUPPORTED_FMT for fmt other than E4M3/E5M2.
+ * Source: "随机舍入" in section "应对FP8训练稳定性挑战的策略" of
+ * "FP8训练的稳定性挑战…" (which fixes no resolution for the draws). */
+int fp8adam_encode_sr16(int32_t fmt, const float* x, const uint32_t* w,
+                        uint8_t* out, int64_t n, void* cuda_stream);
 
 /* out[j] = dec(fmt, codes[j]) as fp32. */
 int fp8adam_decode(int32_t fmt, const uint8_t* codes, float* out, int64_t n,

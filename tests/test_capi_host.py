@@ -154,7 +154,7 @@ def test_option_entry_points_reject_bad_arguments_on_host(L):
     ok = dict(scale_m=8, scale_v=8, amax_m=8, amax_v=8, m_fmt=0, v_fmt=1)
     assert L.fp8adam_create_ex(t, 1, None, ctypes.byref(out)) == capi.ERR_INVALID_ARG
     for bad in (dict(margin_m=-1), dict(margin_v=65), dict(amax_history_len=4), dict(amax_history_len=2000),
-                dict(flags=64), dict(scale_v=0), dict(chunk_elems=100), dict(chunk_elems=1 << 20),
+                dict(flags=64), dict(flags=capi.FLAG_SR_DRAW16), dict(scale_v=0), dict(chunk_elems=100), dict(chunk_elems=1 << 20),
                 dict(chunk_elems=-4096)):
         o = capi.fp8adam_options(**{**ok, **bad})
         assert L.fp8adam_create_ex(t, 1, ctypes.byref(o), ctypes.byref(out)) == capi.ERR_INVALID_ARG, bad

@@ -3,7 +3,8 @@ against the oracle's extended step, free-running from the same seeded state
 on the same seeded gradients.  Covered options:
 - scale margin and amax history;
 - update from stored moments;
-- stochastic rounding;
+- stochastic rounding, with 32-bit draws (integer encoder) and with 16-bit
+  draws (the hardware stochastic-rounding conversion);
 - loss-scale removal, global-norm clipping and skip-on-non-finite;
 - the bf16 param copy."""
 import math
@@ -43,7 +44,8 @@ class ExtRun:
         self.ref = {i: oracle.TensorState(M.view(M.p, i).cpu().numpy(), mf, vf) for i in self.subset}
         self.t = 0
         self.flags = ((oracle.FLAG_UPDATE_FROM_STORED if opt.get("update_from_stored") else 0)
-                      | (oracle.FLAG_STOCHASTIC if opt.get("stochastic_rounding") else 0))
+                      | (oracle.FLAG_STOCHASTIC if opt.get("stochastic_rounding") else 0)
+                      | (oracle.FLAG_SR_DRAW16 if opt.get("sr_draw_bits") == 16 else 0))
 
     def step(self, loss_scale=1.0, max_norm=0.0, skip_nonfinite=False, poison=None, fill=None):
         self.t += 1
@@ -114,24 +116,56 @@ def test_update_from_stored_moments(vf):
         r.compare()
 
 
+DRAWS = pytest.mark.parametrize("draws", [32, 16], ids=["d32", "d16"])
+
+
+@DRAWS
 @pytest.mark.parametrize("tma", [True, False], ids=["staged", "vector"])
 @pytest.mark.parametrize("fmts", [(oracle.E4M3, oracle.E5M2), (oracle.E5M2, oracle.E4M3)], ids=["m4v5", "m5v4"])
-def test_stochastic_rounding(fmts, tma):
-    r = ExtRun(43, mf=fmts[0], vf=fmts[1], stochastic_rounding=True, seed=0x0123456789ABCDEF, tma=tma)
+def test_stochastic_rounding(fmts, tma, draws):
+    """The lean staged kernel (no other option) or the per-thread kernel, on
+    tensors of 0, 33 and ragged sizes among whole ones: codes, params, scales
+    and amax equal the oracle's bit for bit over five steps."""
+    r = ExtRun(43, mf=fmts[0], vf=fmts[1], stochastic_rounding=True, seed=0x0123456789ABCDEF, tma=tma,
+               sr_draw_bits=draws)
     for _ in range(5):
         r.step()
         r.compare()
 
 
-def test_stochastic_rounding_with_a_loss_scale():
+@DRAWS
+def test_stochastic_rounding_with_a_loss_scale(draws):
     """Stochastic rounding with a loss scale and no clipping: the multiplier
     1/loss_scale is a kernel argument, so the staged kernel that keeps the
     multiply runs (the lean one assumes multiplier 1); codes, params, scales
     and amax equal the oracle's bit for bit."""
-    r = ExtRun(54, stochastic_rounding=True, seed=0xABCDEF)
+    r = ExtRun(54, stochastic_rounding=True, seed=0xABCDEF, sr_draw_bits=draws)
     for ls in (4.0, 1000.0, 1.0, 65536.0):
         r.step(loss_scale=ls)
         r.compare()
+
+
+@pytest.mark.parametrize("vf", [oracle.E5M2, oracle.E4M3], ids=["v5", "v4"])
+def test_sr16_with_update_from_stored_and_bf16_copy(vf):
+    """16-bit-draw stochastic rounding in the staged kernel with every option
+    compiled in: the update reads the stored (stochastically rounded) codes
+    and the bf16 copy is written; bit for bit against the oracle."""
+    r = ExtRun(55, vf=vf, bf16=True, update_from_stored=True, stochastic_rounding=True, seed=31337,
+               sr_draw_bits=16, margin_v=1)
+    for _ in range(5):
+        r.step()
+        r.compare()
+
+
+def test_sr16_draw_flag_needs_stochastic_rounding():
+    dev = torch.device("cuda:0")
+    p = [torch.zeros(100, device=dev)]
+    g = [torch.zeros(100, device=dev, dtype=torch.bfloat16)]
+    with pytest.raises(capi.Fp8AdamError) as e:
+        FP8AdamW(p, g, sr_draw_bits=16)
+    assert e.value.code == capi.ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        FP8AdamW(p, g, stochastic_rounding=True, sr_draw_bits=8)
 
 
 @pytest.mark.parametrize("tma", [True, False], ids=["staged", "vector"])
@@ -196,7 +230,8 @@ def test_options_with_fp32_moments_and_current_scaling():
         r.compare()
 
 
-def test_options_on_misaligned_views():
+@DRAWS
+def test_options_on_misaligned_views(draws):
     """Buffers (and the bf16 outputs) that start one element into their
     allocation take the element-by-element path of the staged variant
     kernel; stochastic rounding, a margin, the history and the bf16 copy must
@@ -210,11 +245,11 @@ def test_options_on_misaligned_views():
     pb = [torch.zeros(n + 1, device=dev, dtype=torch.bfloat16)[1:] for n in ns]
     specs = workloads.custom_layout(ns)
     workloads.init_params_into(specs, p, 49)
-    kw = dict(stochastic_rounding=True, seed=99, margin_m=1, amax_history_len=3)
+    kw = dict(stochastic_rounding=True, seed=99, margin_m=1, amax_history_len=3, sr_draw_bits=draws)
     opt = FP8AdamW(p, g, m=m, v=v, param_bf16=pb, **kw)
     ref = [oracle.TensorState(x.cpu().numpy(), oracle.E4M3, oracle.E5M2) for x in p]
     sig = workloads.tensor_sigmas(specs, 49)
-    flags = oracle.FLAG_STOCHASTIC
+    flags = oracle.FLAG_STOCHASTIC | (oracle.FLAG_SR_DRAW16 if draws == 16 else 0)
     for t in range(1, 5):
         workloads.grads_into(specs, g, 49, t, sig)
         opt.step(loss_scale=2.0)
@@ -253,7 +288,8 @@ def test_options_through_host_step():
     a.compare()  # and a against the oracle
 
 
-def test_options_on_the_llama2_100m_layout():
+@DRAWS
+def test_options_on_the_llama2_100m_layout(draws):
     """Stochastic rounding, a 16-step history, margins and the bf16 copy on
     the 110-tensor Llama2-100M layout in the launch configuration the bench
     times (guided chunk table, staged kernel); the embedding, the first and
@@ -261,7 +297,20 @@ def test_options_on_the_llama2_100m_layout():
     specs = workloads.layout("llama2_100m")
     subset = [0, 1, 5, len(specs) - 2, len(specs) - 1]
     r = ExtRun(52, specs=specs, subset=subset, bf16=True, stochastic_rounding=True, seed=77,
-               amax_history_len=16, margin_m=1, margin_v=2)
+               amax_history_len=16, margin_m=1, margin_v=2, sr_draw_bits=draws)
+    for _ in range(3):
+        r.step()
+    r.compare()
+
+
+@DRAWS
+def test_lean_stochastic_rounding_on_the_llama2_100m_layout(draws):
+    """The lean stochastic-rounding kernels (no other option) on the
+    Llama2-100M layout in the bench's launch configuration: the guided chunk
+    table, the staged kernel; a subset of tensors against the oracle."""
+    specs = workloads.layout("llama2_100m")
+    subset = [0, 2, 7, len(specs) - 1]
+    r = ExtRun(56, specs=specs, subset=subset, stochastic_rounding=True, seed=2024, sr_draw_bits=draws)
     for _ in range(3):
         r.step()
     r.compare()
@@ -323,6 +372,33 @@ def test_stochastic_rounding_counter_beyond_2_pow_33():
             xv = np.float32(np.float32(omb2 * np.float32(gj * gj)) * s_v)
             em = oracle.encode_sr(oracle.E4M3, float(xm), oracle.sr_bits(seed, 0, 1, j, 0))
             ev = oracle.encode_sr(oracle.E5M2, float(xv), oracle.sr_bits(seed, 0, 1, j, 1))
+            assert got_m[o] == em and got_v[o] == ev, (j, got_m[o], em, got_v[o], ev)
+        assert (got_p.view(np.uint32) == ref.p[(np.arange(st, st + k) % period)].view(np.uint32)).all()
+    opt.close()
+    # the same step with 16-bit draws on the same buffers (reset in place):
+    # element j's word comes from the call of j/8, whose counter passes 2^30
+    # past element 2^33, and the staged kernel's element indices pass 2^32
+    full = n // period
+    p[:full * period].view(full, period).copy_(pp.to(dev).unsqueeze(0).expand(full, period))
+    p[full * period:].copy_(pp[:n - full * period].to(dev))
+    m.zero_()
+    v.zero_()
+    opt = FP8AdamW([p], [g], m=[m], v=[v], stochastic_rounding=True, sr_draw_bits=16, seed=seed)
+    opt.step()
+    opt.check()
+    assert float(opt.scale_m[0]) == float(ref.scale_m[0]) and float(opt.scale_v[0]) == float(ref.scale_v[0])
+    for st in starts:
+        k = 192
+        got_m = m[st:st + k].cpu().numpy()
+        got_v = v[st:st + k].cpu().numpy()
+        got_p = p[st:st + k].cpu().numpy()
+        for o in range(k):
+            j = st + o
+            gj = gf[j % period]
+            xm = np.float32(np.float32(omb1 * gj) * s_m)
+            xv = np.float32(np.float32(omb2 * np.float32(gj * gj)) * s_v)
+            em = oracle.encode_sr16(oracle.E4M3, float(xm), oracle.sr16_bits(seed, 0, 1, j, 0))
+            ev = oracle.encode_sr16(oracle.E5M2, float(xv), oracle.sr16_bits(seed, 0, 1, j, 1))
             assert got_m[o] == em and got_v[o] == ev, (j, got_m[o], em, got_v[o], ev)
         assert (got_p.view(np.uint32) == ref.p[(np.arange(st, st + k) % period)].view(np.uint32)).all()
     opt.close()
