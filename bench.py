@@ -470,10 +470,11 @@ def our_arm(args):
 
 def ablation_report(args):
     """Moment-format ablation on the Llama2-100M layout ([EXPL] "实验证据
-    (Fig. 5)"): all four (m, v) format pairs and the fp32-moment run, in
-    lockstep on the same seeded gradients.  Per mode: step throughput, the
-    per-step count of v elements flushed to zero, and the per-step max
-    |p_mode - p_fp32| (gradients are open-loop, so the difference is the
+    (Fig. 5)"): all four (m, v) format pairs and the fp32-moment run, plus
+    the four pairs with stochastic rounding on 16-bit draws, in lockstep on
+    the same seeded gradients.  Per mode: step throughput, the
+    per-step count of v elements flushed to zero, and the per-step max and
+    mean |p_mode - p_fp32| (gradients are open-loop, so the difference is the
     optimizer's own error)."""
     import torch
 
@@ -485,22 +486,28 @@ def ablation_report(args):
     specs = workloads.layout(name)
     cfg = workloads.CFG_ID[name]
     n_params = workloads.total_params(specs)
-    modes = {"m4v4": ("e4m3", "e4m3"), "m4v5": ("e4m3", "e5m2"), "m5v4": ("e5m2", "e4m3"),
-             "m5v5": ("e5m2", "e5m2"), "fp32": ("fp32", "fp32")}
+    # (m format, v format, rounding): round to nearest, and stochastic rounding
+    # with 16-bit draws for every FP8 pair
+    modes = {"m4v4": ("e4m3", "e4m3", "rn"), "m4v5": ("e4m3", "e5m2", "rn"), "m5v4": ("e5m2", "e4m3", "rn"),
+             "m5v5": ("e5m2", "e5m2", "rn"), "fp32": ("fp32", "fp32", "rn"),
+             "m4v4_sr16": ("e4m3", "e4m3", "sr16"), "m4v5_sr16": ("e4m3", "e5m2", "sr16"),
+             "m5v4_sr16": ("e5m2", "e4m3", "sr16"), "m5v5_sr16": ("e5m2", "e5m2", "sr16")}
     models, opts = {}, {}
     g = workloads.FlatModel(specs, dev).g  # one gradient buffer shared by all modes
-    for k, (mf, vf) in modes.items():
+    for k, (mf, vf, rnd) in modes.items():
         M = workloads.FlatModel(specs, dev, m_fp32=mf == "fp32", v_fp32=vf == "fp32")
         workloads.init_params_into(specs, M.views(M.p), cfg)
         M.g = g
         models[k] = M
+        sr = dict(stochastic_rounding=True, seed=0xAB1A7E, sr_draw_bits=16) if rnd == "sr16" else {}
         opts[k] = FP8AdamW(M.views(M.p), M.views(g), m_fmt=mf, v_fmt=vf, m=M.views(M.m), v=M.views(M.v),
                            scale_m=M.scale_m, scale_v=M.scale_v, amax_m=M.amax_m, amax_v=M.amax_v,
-                           stats=True)
+                           stats=True, **sr)
     sig = workloads.tensor_sigmas(specs, cfg)
     off = workloads.offsets(specs)
     views = [g[off[i]:off[i] + s.numel] for i, s in enumerate(specs)]
-    out = {k: {"flushed_v": [], "saturated": [], "max_abs_dp_vs_fp32": [], "ms": []} for k in modes}
+    out = {k: {"flushed_v": [], "saturated": [], "max_abs_dp_vs_fp32": [], "mean_abs_dp_vs_fp32": [], "ms": []}
+           for k in modes}
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     for t in range(1, args.steps + 1):
         workloads.grads_into(specs, views, cfg, t, sig)
@@ -515,17 +522,19 @@ def ablation_report(args):
             out[k]["flushed_v"].append(f)
             out[k]["saturated"].append(s_)
         for k in modes:
-            d = (models[k].p - models["fp32"].p).abs().max()
-            out[k]["max_abs_dp_vs_fp32"].append(float(d))
+            d = (models[k].p - models["fp32"].p).abs()
+            out[k]["max_abs_dp_vs_fp32"].append(float(d.max()))
+            out[k]["mean_abs_dp_vs_fp32"].append(float(d.mean(dtype=torch.float64)))
     res = {}
-    for k, (mf, vf) in modes.items():
+    for k, (mf, vf, rnd) in modes.items():
         ms = sorted(out[k]["ms"][3:] or out[k]["ms"])
         med = ms[len(ms) // 2]
         bpp = 4 + 2 + 4 + (8 if mf == "fp32" else 2) + (8 if vf == "fp32" else 2)
-        res[k] = {"m_fmt": mf, "v_fmt": vf, "params_per_s": n_params / (med / 1e3),
+        res[k] = {"m_fmt": mf, "v_fmt": vf, "rounding": rnd, "params_per_s": n_params / (med / 1e3),
                   "gb_per_s": bpp * n_params / (med / 1e3) / 1e9, "bytes_per_param": bpp,
                   "flushed_v_mean": sum(out[k]["flushed_v"]) / args.steps,
-                  "final_max_abs_dp_vs_fp32": out[k]["max_abs_dp_vs_fp32"][-1], **out[k]}
+                  "final_max_abs_dp_vs_fp32": out[k]["max_abs_dp_vs_fp32"][-1],
+                  "final_mean_abs_dp_vs_fp32": out[k]["mean_abs_dp_vs_fp32"][-1], **out[k]}
         del res[k]["ms"]
     for k, o in opts.items():
         o.check()  # raises if a kernel's bounded wait ran out: no report from a broken run

@@ -266,12 +266,13 @@ def test_options_on_misaligned_views(draws):
         assert (pb[i].cpu().view(torch.int16).numpy().view(np.uint16) == rs.p_bf16).all(), i
 
 
-def test_options_through_host_step():
+@DRAWS
+def test_options_through_host_step(draws):
     """fp8adam_step_host with options: the history and stochastic rounding
     (grouped steps), then loss scale and clipping (one group after all
     copies); the same results as copying the gradients and fp8adam_step_ex."""
-    a = ExtRun(50, amax_history_len=3, stochastic_rounding=True, seed=7)
-    b = ExtRun(50, amax_history_len=3, stochastic_rounding=True, seed=7)
+    a = ExtRun(50, amax_history_len=3, stochastic_rounding=True, seed=7, sr_draw_bits=draws)
+    b = ExtRun(50, amax_history_len=3, stochastic_rounding=True, seed=7, sr_draw_bits=draws)
     h = torch.empty(b.M.g.numel(), dtype=torch.bfloat16, pin_memory=True)
     views = [h[o:o + s.numel] for o, s in zip(b.M.off, b.specs)]
     for t in range(1, 6):
@@ -314,6 +315,22 @@ def test_lean_stochastic_rounding_on_the_llama2_100m_layout(draws):
     for _ in range(3):
         r.step()
     r.compare()
+
+
+@pytest.mark.slow
+@DRAWS
+def test_stochastic_rounding_60_steps_on_the_llama2_100m_layout(draws):
+    """Free-running stochastic rounding (lean kernels) over 60 steps of the
+    Llama2-100M layout: the embedding, a projection, a norm gain and the last
+    matrix against the oracle, bit for bit, at steps 1, 20, 40 and 60."""
+    specs = workloads.layout("llama2_100m")
+    subset = [0, 3, 6, len(specs) - 2]
+    r = ExtRun(57, specs=specs, subset=subset, stochastic_rounding=True, seed=0xFEED, sr_draw_bits=draws)
+    for t in range(1, 61):
+        r.step()
+        if t in (1, 20, 40, 60):
+            r.compare()
+    r.opt.check()
 
 
 @pytest.mark.slow
