@@ -419,3 +419,24 @@ def test_stochastic_rounding_counter_beyond_2_pow_33():
             assert got_m[o] == em and got_v[o] == ev, (j, got_m[o], em, got_v[o], ev)
         assert (got_p.view(np.uint32) == ref.p[(np.arange(st, st + k) % period)].view(np.uint32)).all()
     opt.close()
+
+
+@DRAWS
+def test_stochastic_rounding_does_not_depend_on_the_chunk_table(draws):
+    """Each element's draw is a function of its index, tensor and step alone,
+    so chunk lengths of 4K, 64K and 128K elements and the guided table (and
+    with them the staged kernel's pairing of threads) give the same codes and
+    params, bit for bit, over four steps."""
+    outs = []
+    for chunk in (4096, 65536, 131072, 0):
+        r = ExtRun(58, sizes=[70001, 4096, 33, 3 * 65536 + 4099, 200003], stochastic_rounding=True, seed=11,
+                   sr_draw_bits=draws, chunk_elems=chunk, subset=[])
+        for _ in range(4):
+            r.step()
+        torch.cuda.synchronize()
+        outs.append([x.clone() for x in (r.M.p, r.M.m, r.M.v, r.M.scale_m, r.M.scale_v, r.M.amax_m, r.M.amax_v)])
+        r.opt.check()
+        r.opt.close()
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))

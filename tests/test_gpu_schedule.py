@@ -72,8 +72,9 @@ def test_learning_rate_schedule_against_the_oracle():
 
 
 @pytest.mark.parametrize("opts", [{}, dict(stochastic_rounding=True, seed=5, amax_history_len=4, margin_v=1),
+                                  dict(stochastic_rounding=True, sr_draw_bits=16, seed=5, amax_history_len=4),
                                   dict(tma=False), dict(tma=False, stochastic_rounding=True, seed=5, amax_history_len=4)],
-                         ids=["default", "sr_history_margin", "vector", "vector_sr_history"])
+                         ids=["default", "sr_history_margin", "sr16_history", "vector", "vector_sr_history"])
 def test_captured_graph_replays_equal_regular_steps(opts):
     """One fp8adam_step_scheduled captured in a CUDA graph, replayed once per
     step with new gradients written between replays, against fp8adam_step_ex
