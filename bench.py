@@ -164,12 +164,13 @@ def single_thread_specs(specs, idx):
     return out
 
 
-def run_oracle_sample(name: str, steps: int, warmup: int, single_thread: bool = False):
+def run_oracle_sample(name: str, steps: int, warmup: int, single_thread: bool = False, variant: str = "default"):
     """Times the CPU oracle, as it stands, on a sample of the layout: one host
     thread per tensor on every available core (ctypes releases the GIL), or
-    one thread in all.  Steps after the first are steady-state (t > 1).
-    Returns (params/s, ms per step of the sample, threads used, sample
-    description)."""
+    one thread in all.  Steps after the first are steady-state (t > 1).  A
+    variant runs the oracle's extended step with the variant's options (for
+    clipping, the multiplier from the sample's own gradients).  Returns
+    (params/s, ms per step of the sample, threads used, sample description)."""
     from concurrent.futures import ThreadPoolExecutor
 
     import numpy as np
@@ -196,9 +197,27 @@ def run_oracle_sample(name: str, steps: int, warmup: int, single_thread: bool = 
     n = sum(s.numel for s in sub)
     order = sorted(range(len(sub)), key=lambda k: -sub[k].numel)
 
+    ex_kw, ex_flags = {}, 0
+    if variant in ("sr", "sr16"):
+        ex_flags = oracle.FLAG_STOCHASTIC | (oracle.FLAG_SR_DRAW16 if variant == "sr16" else 0)
+        ex_kw = dict(seed=1234)
+    elif variant == "history":
+        ex_kw = dict(hist_len=16)
+    elif variant == "jit":
+        ex_flags = oracle.FLAG_JIT_EVERY_STEP
+
     def step(t):
+        gm = 1.0
+        if variant == "clip":  # loss scale 1024, clip to 1.0: the multiplier from the sample's sum of squares
+            sumsq, _ = oracle.grad_sumsq(grads)
+            gm = oracle.grad_multiplier(sumsq, 1024.0, 1.0)
+
         def one(k):
-            states[k].step(grads[k], hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], t)
+            if variant == "default":
+                states[k].step(grads[k], hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], t)
+            else:
+                states[k].step_ex(grads[k], hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], t,
+                                  ex_flags, tensor_index=idx[k], grad_mult=gm, **ex_kw)
         with ThreadPoolExecutor(threads) as ex:
             list(ex.map(one, order))
 
@@ -213,17 +232,19 @@ def run_oracle_sample(name: str, steps: int, warmup: int, single_thread: bool = 
         step(t)
         times.append(time.perf_counter() - t0)
     ms = 1e3 * sum(times) / len(times)
-    desc = "%s of the %s layout (%d tensors, %d params), steady-state step (t>1), %d host thread%s" % (
+    desc = "%s of the %s layout (%d tensors, %d params), steady-state step (t>1)%s, %d host thread%s" % (
         "first tensors of layers 0-1" if single_thread else "layers 0-1 (or the first tensors)",
-        name, len(sub), n, threads, "" if threads == 1 else "s, one per tensor")
+        name, len(sub), n, "" if variant == "default" else ", variant " + variant, threads,
+        "" if threads == 1 else "s, one per tensor")
     return n / (ms / 1e3), ms, threads, desc
 
 
-def cpu_baseline(name: str, steps: int = 1, warmup: int = 1) -> dict:
+def cpu_baseline(name: str, steps: int = 1, warmup: int = 1, variant: str = "default") -> dict:
     """The oracle on every available core (the baseline's value) and on one
-    thread, each on its own bounded sample of the layout."""
-    value, ms, threads, desc = run_oracle_sample(name, steps, warmup)
-    v1, ms1, _, desc1 = run_oracle_sample(name, steps, warmup, single_thread=True)
+    thread, each on its own bounded sample of the layout, with the timed
+    variant's options."""
+    value, ms, threads, desc = run_oracle_sample(name, steps, warmup, variant=variant)
+    v1, ms1, _, desc1 = run_oracle_sample(name, steps, warmup, single_thread=True, variant=variant)
     return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
             "sample_ms_per_step": ms, "host_cores": len(os.sched_getaffinity(0)),
             "single_thread": {"value": v1, "unit": UNIT, "cores": 1, "sample": desc1, "sample_ms_per_step": ms1}}
@@ -454,7 +475,7 @@ def our_arm(args):
         import oracle
 
         oracle.build()
-        cpu = cpu_baseline(name)
+        cpu = cpu_baseline(name, variant=args.variant)
 
     opt.close()
     if rank == 0:
