@@ -46,7 +46,7 @@ class fp8adam_options(ctypes.Structure):
                 ("flags", ctypes.c_uint32), ("margin_m", ctypes.c_int32), ("margin_v", ctypes.c_int32),
                 ("amax_history_len", ctypes.c_int32), ("amax_history_m", ctypes.c_void_p),
                 ("amax_history_v", ctypes.c_void_p), ("seed", ctypes.c_uint64), ("param_bf16", ctypes.c_void_p),
-                ("chunk_elems", ctypes.c_int32)]
+                ("chunk_elems", ctypes.c_int32), ("sr_counter_ids", ctypes.c_void_p)]
 
 
 class fp8adam_step_params(ctypes.Structure):

@@ -314,6 +314,7 @@ struct fp8adam_ctx {
   float *hist_m = nullptr, *hist_v = nullptr;
   uint64_t seed = 0;
   uint16_t** d_bf16 = nullptr;  // device [T] bf16 outputs, or null
+  uint32_t* d_sr_ids = nullptr; // device [T] SR counter words of the tensors, or null (their indices)
   bool ext = false;             // any option on: the variant kernels run
   bool tma = false;             // default step through the TMA-staged kernel
   uint32_t* d_error = nullptr;  // device error word (bounded waits that ran out)
@@ -354,6 +355,7 @@ static void free_ctx(fp8adam_ctx* c) {
   cudaFree(c->d_cdesc);
   cudaFree(c->d_error);
   cudaFree(c->d_bf16);
+  cudaFree(c->d_sr_ids);
   cudaFree(c->d_partial);
   cudaFree(c->d_nonfinite);
   cudaFree(c->d_grad_mult);
@@ -596,7 +598,8 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
       cudaMalloc(&c->d_skip, sizeof(uint32_t)) != cudaSuccess ||
       cudaMalloc(&c->d_norm, sizeof(double)) != cudaSuccess ||
       cudaMalloc(&c->d_error, sizeof(uint32_t)) != cudaSuccess ||
-      (opts->param_bf16 && cudaMalloc(&c->d_bf16, T * sizeof(uint16_t*)) != cudaSuccess)) {
+      (opts->param_bf16 && cudaMalloc(&c->d_bf16, T * sizeof(uint16_t*)) != cudaSuccess) ||
+      (opts->sr_counter_ids && cudaMalloc(&c->d_sr_ids, T * sizeof(uint32_t)) != cudaSuccess)) {
     cudaGetLastError();
     free_ctx(c);
     return FP8ADAM_ERR_OOM;
@@ -620,6 +623,8 @@ extern "C" int fp8adam_create_ex(const fp8adam_tensor* tensors, int32_t num_tens
       cudaMemset(c->d_norm, 0, sizeof(double)) != cudaSuccess ||
       (opts->param_bf16 &&
        cudaMemcpy(c->d_bf16, opts->param_bf16, T * sizeof(uint16_t*), cudaMemcpyHostToDevice) != cudaSuccess) ||
+      (opts->sr_counter_ids &&
+       cudaMemcpy(c->d_sr_ids, opts->sr_counter_ids, T * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess) ||
       cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     free_ctx(c);
@@ -746,6 +751,7 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
   e.grad_mult = nullptr;
   e.skip = nullptr;
   e.p_bf16 = ctx->d_bf16;
+  e.sr_ids = (ctx->flags & FP8ADAM_FLAG_STOCHASTIC_ROUNDING) ? ctx->d_sr_ids : nullptr;
   if (prepass) {
     NvtxRange pre("fp8adam grad-norm pre-pass");
     if (cudaMemsetAsync(ctx->d_nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)

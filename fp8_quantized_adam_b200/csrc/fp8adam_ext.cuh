@@ -49,6 +49,7 @@ struct ExtArgs {
   float gm_const;           // gradient multiplier without a pre-pass: 1/loss_scale (1.0: none)
   const uint32_t* skip;     // device flag, or null
   uint16_t* const* p_bf16;  // device array [T] of bf16 outputs (entries may be null), or null
+  const uint32_t* sr_ids;   // device array [T]: each tensor's word in the SR counter, or null (its index)
 };
 
 // ------------------------------------------------------------ Philox4x32-10
@@ -62,10 +63,12 @@ __device__ __forceinline__ uint4 philox_round(uint4 c, uint32_t k0, uint32_t k1)
   return make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ k0, (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ k1, (uint32_t)p0);
 }
 
-// random words of elements (2q, 2q+1) of tensor ti at this step:
-// .x/.y -> element 2q (m, v); .z/.w -> element 2q+1 (m, v)
-__device__ __forceinline__ uint4 sr_words(const ExtArgs& a, int ti, uint32_t t_lo, int64_t q) {
-  uint4 c = make_uint4((uint32_t)q, (uint32_t)((uint64_t)q >> 32), (uint32_t)ti, t_lo);
+// The random words of counter (q, tensor id, step): with 32-bit draws those
+// of elements (2q, 2q+1) (.x/.y: m/v of 2q, .z/.w: of 2q+1), with 16-bit
+// draws those of elements 8q .. 8q+7.  `id` is the tensor's counter word
+// (ExtArgs::sr_ids, by default its index in the table).
+__device__ __forceinline__ uint4 sr_words(const ExtArgs& a, uint32_t id, uint32_t t_lo, int64_t q) {
+  uint4 c = make_uint4((uint32_t)q, (uint32_t)((uint64_t)q >> 32), id, t_lo);
 #pragma unroll
   for (int r = 0; r < 10; ++r) c = philox_round(c, a.sr_key[r][0], a.sr_key[r][1]);
   return c;
@@ -78,8 +81,8 @@ __device__ __forceinline__ uint4 sr_words(const ExtArgs& a, int ti, uint32_t t_l
 struct SrChunk {
   uint32_t x1, y1, w1;
 };
-__device__ __forceinline__ SrChunk sr_chunk(const ExtArgs& a, int ti, uint32_t t_lo, int64_t q0) {
-  const uint64_t p1 = (uint64_t)kPhiloxM1 * (uint32_t)ti;
+__device__ __forceinline__ SrChunk sr_chunk(const ExtArgs& a, uint32_t id, uint32_t t_lo, int64_t q0) {
+  const uint64_t p1 = (uint64_t)kPhiloxM1 * id;
   SrChunk u;
   u.x1 = (uint32_t)(p1 >> 32) ^ (uint32_t)((uint64_t)q0 >> 32) ^ a.sr_key[0][0];
   u.y1 = (uint32_t)p1;
@@ -227,6 +230,7 @@ struct ExtSeg {  // per tensor segment
   float inv_s_m, inv_s_v, s_m_new, s_v_new, inv_s_m_new, inv_s_v_new, gm;
   uint16_t* pb;
   int ti;
+  uint32_t sr_id;     // the tensor's word in the SR counter
   uint32_t t_lo;      // the step, for the SR counter
   int32_t hist_slot;  // this step's slot of the amax history ring
 };
@@ -240,11 +244,11 @@ __device__ __forceinline__ void ext_element(const ExtArgs& a, const TensorDesc& 
   uint32_t rm = 0, rv = 0;
   const int srk = sr_kind<SRM>(a);
   if (srk == 1) {
-    const uint4 r = sr_words(a, sg.ti, sg.t_lo, i >> 1);
+    const uint4 r = sr_words(a, sg.sr_id, sg.t_lo, i >> 1);
     rm = (i & 1) ? r.z : r.x;
     rv = (i & 1) ? r.w : r.y;
   } else if (srk == 2) {
-    const uint4 r = sr_words(a, sg.ti, sg.t_lo, i >> 3);
+    const uint4 r = sr_words(a, sg.sr_id, sg.t_lo, i >> 3);
     rm = ((i >> 2) & 1) ? r.z : r.x;
     rv = ((i >> 2) & 1) ? r.w : r.y;
   }
@@ -291,12 +295,12 @@ __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& 
     uint32_t rmj[4] = {0, 0, 0, 0}, rvj[4] = {0, 0, 0, 0};
     const int srk = sr_kind<SRM>(a);
     if (srk == 1) {
-      const uint4 r0 = sr_words(a, sg.ti, sg.t_lo, (i + 4 * k) >> 1);
-      const uint4 r1 = sr_words(a, sg.ti, sg.t_lo, ((i + 4 * k) >> 1) + 1);
+      const uint4 r0 = sr_words(a, sg.sr_id, sg.t_lo, (i + 4 * k) >> 1);
+      const uint4 r1 = sr_words(a, sg.sr_id, sg.t_lo, ((i + 4 * k) >> 1) + 1);
       rmj[0] = r0.x; rmj[1] = r0.z; rmj[2] = r1.x; rmj[3] = r1.z;
       rvj[0] = r0.y; rvj[1] = r0.w; rvj[2] = r1.y; rvj[3] = r1.w;
     } else if (srk == 2) {  // i + 4k is a multiple of 4: one word for the four m codes, one for the v codes
-      const uint4 r = sr_words(a, sg.ti, sg.t_lo, (i + 4 * k) >> 3);
+      const uint4 r = sr_words(a, sg.sr_id, sg.t_lo, (i + 4 * k) >> 3);
       const bool second = (((i + 4 * k) >> 2) & 1) != 0;
       rmj[0] = rmj[1] = rmj[2] = rmj[3] = second ? r.z : r.x;
       rvj[0] = rvj[1] = rvj[2] = rvj[3] = second ? r.w : r.y;
@@ -342,6 +346,7 @@ __device__ __forceinline__ ExtSeg ext_setup(const ExtArgs& a, int ti, float gm) 
   const StepArgs& S = a.s;
   ExtSeg sg;
   sg.ti = ti;
+  sg.sr_id = a.sr_ids ? a.sr_ids[ti] : (uint32_t)ti;
   sg.gm = gm;
   if (S.cur != nullptr) {  // a scheduled step (the kernel checked that the entry is valid)
     sg.c = S.cur->c;

@@ -166,8 +166,8 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   uint32_t flushed = 0, sat = 0;
 
   SrChunk su{0u, 0u, 0u};
-  if constexpr (SRK == 1) su = sr_chunk(a, ti, sg.t_lo, e0 >> 1);
-  if constexpr (SRK == 2) su = sr_chunk(a, ti, sg.t_lo, e0 >> 3);
+  if constexpr (SRK == 1) su = sr_chunk(a, sg.sr_id, sg.t_lo, e0 >> 1);
+  if constexpr (SRK == 2) su = sr_chunk(a, sg.sr_id, sg.t_lo, e0 >> 3);
   uint32_t w1m = 0, w1v = 0;  // 16-bit draws: the words of this thread's second group of the stage
   if (!tma_run(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
         uint32_t wm = 0, wv = 0;

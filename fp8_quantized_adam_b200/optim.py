@@ -35,7 +35,10 @@ class FP8AdamW:
     allocated here and checkpointed), ``update_from_stored`` (the update reads
     the requantised moments), ``stochastic_rounding`` with ``seed`` and
     ``sr_draw_bits`` (32: the integer encoder with 32-bit draws; 16: 16-bit
-    draws rounded by the hardware's stochastic-rounding conversion), and
+    draws rounded by the hardware's stochastic-rounding conversion) and
+    ``sr_tensor_ids`` (each tensor's word in the random counter, by default
+    its position in ``params``; a shard of a larger model passes the
+    tensors' indices in the whole model), and
     ``param_bf16`` (bf16 tensors receiving the updated params).  Per step:
     ``step(loss_scale=, max_norm=, skip_nonfinite=)`` (fp8adam_step_ex).
     """
@@ -49,6 +52,7 @@ class FP8AdamW:
                  jit_every_step: bool = False, margin_m: int = 0, margin_v: int = 0,
                  amax_history_len: int = 0, update_from_stored: bool = False,
                  stochastic_rounding: bool = False, seed: int = 0, sr_draw_bits: int = 32,
+                 sr_tensor_ids: Optional[Sequence[int]] = None,
                  param_bf16: Optional[List[torch.Tensor]] = None, chunk_elems: int = 0,
                  tma: bool = True):
         if len(params) == 0 or len(params) != len(grads):
@@ -119,13 +123,18 @@ class FP8AdamW:
         if self.param_bf16 is not None:
             check(self.param_bf16, torch.bfloat16, "param_bf16")
             bf16_arr = (ctypes.c_void_p * T)(*[b.data_ptr() for b in self.param_bf16])
+        ids_arr = None
+        if sr_tensor_ids is not None:
+            if len(sr_tensor_ids) != T or any(not 0 <= int(i) < (1 << 32) for i in sr_tensor_ids):
+                raise ValueError("sr_tensor_ids: one 32-bit unsigned id per tensor")
+            ids_arr = (ctypes.c_uint32 * T)(*[int(i) for i in sr_tensor_ids])
         opts = capi.fp8adam_options(self.scale_m.data_ptr(), self.scale_v.data_ptr(), self.amax_m.data_ptr(),
                                     self.amax_v.data_ptr(), self.m_fmt, self.v_fmt, flags, margin_m, margin_v,
                                     self.amax_history_len,
                                     self.hist_m.data_ptr() if self.hist_m is not None else None,
                                     self.hist_v.data_ptr() if self.hist_v is not None else None,
                                     seed, ctypes.cast(bf16_arr, ctypes.c_void_p) if bf16_arr is not None else None,
-                                    chunk_elems)
+                                    chunk_elems, ctypes.cast(ids_arr, ctypes.c_void_p) if ids_arr is not None else None)
         with torch.cuda.device(dev):
             self.ctx = capi.fp8adam_create_ex(arr, T, opts)
         self.device = dev

@@ -123,6 +123,10 @@ class ZeroFP8AdamW:
             from .optim import FP8AdamW
 
             make_local = lambda p, g, **kw: FP8AdamW(p, g, **kw)  # noqa: E731
+        # each owned tensor keeps its index in the whole model as its word in
+        # the stochastic-rounding counter, so a shard draws the bits a single
+        # optimizer over every tensor would
+        opt_kw.setdefault("sr_tensor_ids", list(layout.parts[r]))
         self.local = make_local(p_views, g_views, **opt_kw) if p_views else None
 
     def step(self, **step_kw) -> None:

@@ -211,9 +211,11 @@ typedef struct {
   uint64_t seed;             /* stochastic rounding: random bits of element j of
                                 tensor i at step t for moment w (0 = m, 1 = v) are
                                 word 2*(j&1) + w of Philox4x32-10 with counter
-                                (j/2 low, j/2 high, i, t low 32 bits) and key
+                                (j/2 low, j/2 high, id(i), t low 32 bits) and key
                                 (seed low, seed high); a code rounds up to the
-                                next grid value iff r*(hi-lo) < (|x|-lo)*2^32 */
+                                next grid value iff r*(hi-lo) < (|x|-lo)*2^32
+                                (16-bit draws: FP8ADAM_FLAG_SR_DRAW16).  id(i)
+                                is sr_counter_ids[i], or i. */
   uint16_t* const* param_bf16; /* host array [num_tensors] of device bf16 buffers
                                   [numel] receiving the updated params rounded to
                                   nearest even (entries may be NULL), or NULL */
@@ -228,6 +230,14 @@ typedef struct {
                                 one that would cross a multiple of 2^33
                                 elements of its tensor, is cut shorter.
                                 Results do not depend on it. */
+  const uint32_t* sr_counter_ids; /* host array [num_tensors], read by create:
+                                tensor i's word in the stochastic-rounding
+                                counter (id(i) above), e.g. its index in a model
+                                whose tensors are split over several contexts
+                                (ZeRO-1 shards), so that every tensor draws the
+                                same bits as in one context over the whole
+                                model; NULL: i.  Any values; tensors sharing an
+                                id and a seed share their draws. */
 } fp8adam_options;
 
 /* fp8adam_create with options (fp8adam_create is this call with the options

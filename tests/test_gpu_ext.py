@@ -69,7 +69,8 @@ class ExtRun:
             r.step_ex(grads[i], HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], self.t,
                       self.flags, margin_m=self.opt_kw.get("margin_m", 0), margin_v=self.opt_kw.get("margin_v", 0),
                       hist_len=self.opt_kw.get("amax_history_len", 0), seed=self.opt_kw.get("seed", 0),
-                      tensor_index=i, grad_mult=gm, skip=skip, want_bf16=self.bf16 is not None)
+                      tensor_index=self.opt_kw.get("sr_tensor_ids", range(len(self.specs)))[i], grad_mult=gm,
+                      skip=skip, want_bf16=self.bf16 is not None)
         return norm, skip
 
     def compare(self):
@@ -440,3 +441,19 @@ def test_stochastic_rounding_does_not_depend_on_the_chunk_table(draws):
     for o in outs[1:]:
         for a, b in zip(outs[0], o):
             assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+
+
+@DRAWS
+def test_sr_tensor_ids_key_the_draws(draws):
+    """Caller-given counter words (sr_tensor_ids): tensor i draws as the
+    oracle's tensor ids[i] (here large, out of order, and one shared), bit for
+    bit, over three steps; without them the codes differ."""
+    ids = [7, 1 << 31, 3, 99, 3, 0xFFFFFFFF]
+    r = ExtRun(59, stochastic_rounding=True, seed=4242, sr_draw_bits=draws, sr_tensor_ids=ids)
+    plain = ExtRun(59, stochastic_rounding=True, seed=4242, sr_draw_bits=draws, subset=[])
+    for _ in range(3):
+        r.step()
+        plain.step()
+        r.compare()
+    torch.cuda.synchronize()
+    assert not torch.equal(r.M.m, plain.M.m)

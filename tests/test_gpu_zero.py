@@ -53,7 +53,16 @@ def test_zero1_single_rank_nccl_matches_oracle():
 SIZES2 = [70001, 4096, 33, 200003, 5000, 1, 0, 131072 * 2 + 77]
 
 
-def _two_rank_worker(rank, world, port, q):
+SR2 = {"rn": {}, "sr16": dict(stochastic_rounding=True, sr_draw_bits=16, seed=0xBEEF)}
+
+
+def _sr_flags(kw):
+    if not kw.get("stochastic_rounding"):
+        return 0
+    return oracle.FLAG_STOCHASTIC | (oracle.FLAG_SR_DRAW16 if kw.get("sr_draw_bits") == 16 else 0)
+
+
+def _two_rank_worker(rank, world, port, q, sr):
     """One rank: the real CUDA step on its shard (cuda:0, shared with the
     other rank), collectives on host copies over gloo."""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank),
@@ -73,7 +82,8 @@ def _two_rank_worker(rank, world, port, q):
         p0 = params.cpu()
         grads = torch.zeros(L.total, dtype=torch.bfloat16, device=dev)
         opt = zero.ZeroFP8AdamW(L, params, grads, collectives=zero.HostCollectives(), lr=HP["lr"],
-                                betas=(HP["beta1"], HP["beta2"]), eps=HP["eps"], weight_decay=HP["weight_decay"])
+                                betas=(HP["beta1"], HP["beta2"]), eps=HP["eps"], weight_decay=HP["weight_decay"],
+                                **sr)
         sig = workloads.tensor_sigmas(specs, 71)
         reduced = []
         launches0 = capi.fp8adam_launch_count()
@@ -90,9 +100,9 @@ def _two_rank_worker(rank, world, port, q):
         c = oracle.grad_multiplier(0.0, float(world), 0.0)
         ref = [oracle.TensorState(v.numpy(), oracle.E4M3, oracle.E5M2) for v in L.views(p0)]
         for t, full in enumerate(reduced, start=1):
-            for st, g in zip(ref, L.views(full)):
+            for i, (st, g) in enumerate(zip(ref, L.views(full))):
                 st.step_ex(bf16_host_bits(g), HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], t,
-                           grad_mult=c)
+                           _sr_flags(sr), grad_mult=c, seed=sr.get("seed", 0), tensor_index=i)
         ph = params.cpu()
         ok = all((v.numpy().view(np.uint32) == st.p.view(np.uint32)).all() for v, st in zip(L.views(ph), ref))
         # this rank's moments, scales and amax
@@ -110,7 +120,8 @@ def _two_rank_worker(rank, world, port, q):
         q.put((rank, False, repr(ex), -1))
 
 
-def test_zero1_two_gloo_ranks_run_the_cuda_step():
+@pytest.mark.parametrize("sr", list(SR2))
+def test_zero1_two_gloo_ranks_run_the_cuda_step(sr):
     """ZeRO-1 at world size 2 with the CUDA step inside it: two processes
     share cuda:0, each runs FP8AdamW on the tensors it owns between a real
     reduce-scatter and all-gather (gloo, on host copies; the ranks' kernels
@@ -118,14 +129,16 @@ def test_zero1_two_gloo_ranks_run_the_cuda_step():
     and each rank's moment codes, scales and amax, equal a single-process
     oracle run over all tensors on the summed gradients, bit for bit.  The
     1/world average is a constant multiplier: one step kernel per step after
-    step 1, no gradient pre-pass."""
+    step 1, no gradient pre-pass.  With stochastic rounding (16-bit draws)
+    each shard keys its draws by the tensors' indices in the whole model, so
+    the sharded run still equals the single-process one."""
     import torch.multiprocessing as mp
 
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    ps = [ctx.Process(target=_two_rank_worker, args=(r, world, port, q)) for r in range(world)]
+    ps = [ctx.Process(target=_two_rank_worker, args=(r, world, port, q, SR2[sr])) for r in range(world)]
     for p in ps:
         p.start()
     res = [q.get(timeout=600) for _ in range(world)]

@@ -5,7 +5,9 @@ partition, rank-blocked flat buffers, reduce-scatter of the gradients,
 the step on owned tensors only, and the all-gather of the params.  The local
 step is the CPU oracle, a test stand-in for the CUDA kernels; the product's
 local step is FP8AdamW.  After three steps every rank's params must equal a
-single-process oracle run over all tensors on the summed gradients.
+single-process oracle run over all tensors on the summed gradients; with
+stochastic rounding too, since each shard passes its tensors' indices in the
+whole model as their words in the random counter.
 """
 import os
 import socket
@@ -26,25 +28,34 @@ def _bits(t):
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
+def _sr_flags(stochastic_rounding=False, sr_draw_bits=32, **_):
+    if not stochastic_rounding:
+        return 0
+    return oracle.FLAG_STOCHASTIC | (oracle.FLAG_SR_DRAW16 if sr_draw_bits == 16 else 0)
+
+
 class OracleLocal:
     """CPU stand-in for FP8AdamW over the owned tensors (views are updated in
-    place so the all-gather sees the new params)."""
+    place so the all-gather sees the new params); takes FP8AdamW's
+    stochastic-rounding options, the tensor ids included."""
 
-    def __init__(self, p_views, g_views, **kw):
+    def __init__(self, p_views, g_views, sr_tensor_ids=None, seed=0, **kw):
         self.p, self.g = p_views, g_views
         self.st = [oracle.TensorState(p.numpy(), oracle.E4M3, oracle.E5M2) for p in p_views]
+        self.ids = list(sr_tensor_ids) if sr_tensor_ids is not None else list(range(len(p_views)))
+        self.flags, self.seed = _sr_flags(**kw), seed
         self.t = 0
 
     def step(self, loss_scale=1.0, **kw):
         self.t += 1
         c = oracle.grad_multiplier(0.0, loss_scale, 0.0)
-        for p, g, st in zip(self.p, self.g, self.st):
+        for p, g, st, tid in zip(self.p, self.g, self.st, self.ids):
             st.step_ex(_bits(g), HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], self.t,
-                       grad_mult=c)
+                       self.flags, grad_mult=c, seed=self.seed, tensor_index=tid)
             p.copy_(torch.from_numpy(st.p))
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, sr):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank),
                       LOCAL_RANK=str(rank))
     import torch.distributed as dist
@@ -56,7 +67,7 @@ def _worker(rank, world, port, q):
     workloads.init_params_into(specs, L.views(params), 51)  # identical on every rank
     p0 = params.clone()
     grads = torch.zeros(L.total, dtype=torch.bfloat16)
-    opt = zero.ZeroFP8AdamW(L, params, grads, make_local=OracleLocal)
+    opt = zero.ZeroFP8AdamW(L, params, grads, make_local=OracleLocal, **sr)
     sig = workloads.tensor_sigmas(specs, 51)
     reduced = []
     for t in range(1, 4):
@@ -70,9 +81,9 @@ def _worker(rank, world, port, q):
         c = oracle.grad_multiplier(0.0, float(world), 0.0)
         ref = [oracle.TensorState(v.numpy(), oracle.E4M3, oracle.E5M2) for v in L.views(p0)]
         for t, full in enumerate(reduced, start=1):
-            for st, g in zip(ref, L.views(full)):
+            for i, (st, g) in enumerate(zip(ref, L.views(full))):
                 st.step_ex(_bits(g), HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], t,
-                           grad_mult=c)
+                           _sr_flags(**sr), grad_mult=c, seed=sr.get("seed", 0), tensor_index=i)
         ok = all((v.numpy().view(np.uint32) == st.p.view(np.uint32)).all() for v, st in zip(L.views(params), ref))
         q.put(("rank0", ok, [len(p) for p in L.parts]))
     else:
@@ -86,12 +97,19 @@ def _free_port():
         return s.getsockname()[1]
 
 
+SR = {"rn": {}, "sr16": dict(stochastic_rounding=True, sr_draw_bits=16, seed=0xC0FFEE),
+      "sr32": dict(stochastic_rounding=True, seed=0xC0FFEE)}
+
+
+@pytest.mark.parametrize("sr", list(SR))
 @pytest.mark.parametrize("world", [2, 3])
-def test_zero1_matches_single_process_oracle(world):
+def test_zero1_matches_single_process_oracle(world, sr):
+    if sr == "sr32" and world == 3:
+        pytest.skip("one world size suffices for the 32-bit draws")
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    ps = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    ps = [ctx.Process(target=_worker, args=(r, world, port, q, SR[sr])) for r in range(world)]
     for p in ps:
         p.start()
     res = dict((k, (ok, parts)) for k, ok, parts in (q.get(timeout=300) for _ in range(world)))
