@@ -99,9 +99,12 @@ class HostCollectives(TorchCollectives):
 class ZeroFP8AdamW:
     """ZeRO-1 FP8-moment AdamW.  ``params`` (fp32) and ``grads`` (bf16) are
     the rank-blocked flat buffers of a ShardLayout (``layout.views`` gives the
-    per-tensor views a model would use).  ``local_step`` builds the optimizer
-    of the owned shard; by default the CUDA FP8AdamW.  ``collectives``:
-    TorchCollectives (the default: NCCL on CUDA tensors) or HostCollectives."""
+    per-tensor views a model would use).  ``make_local(p_views, g_views,
+    **opt_kw)`` builds the optimizer of the owned shard (by default the CUDA
+    FP8AdamW); besides the caller's options it receives ``sr_tensor_ids``,
+    the owned tensors' indices in the whole model, which key their
+    stochastic-rounding draws.  ``collectives``: TorchCollectives (the
+    default: NCCL on CUDA tensors) or HostCollectives."""
 
     def __init__(self, layout: ShardLayout, params: torch.Tensor, grads: torch.Tensor, *,
                  group=None, make_local: Optional[Callable] = None, collectives=None, **opt_kw):
