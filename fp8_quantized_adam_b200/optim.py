@@ -123,6 +123,10 @@ class FP8AdamW:
         if self.param_bf16 is not None:
             check(self.param_bf16, torch.bfloat16, "param_bf16")
             bf16_arr = (ctypes.c_void_p * T)(*[b.data_ptr() for b in self.param_bf16])
+        # the stochastic-rounding stream: part of the checkpointed state's identity
+        self.sr_config = {"stochastic_rounding": bool(stochastic_rounding), "seed": int(seed),
+                          "sr_draw_bits": int(sr_draw_bits),
+                          "sr_tensor_ids": None if sr_tensor_ids is None else [int(i) for i in sr_tensor_ids]}
         ids_arr = None
         if sr_tensor_ids is not None:
             if len(sr_tensor_ids) != T or any(not 0 <= int(i) < (1 << 32) for i in sr_tensor_ids):
@@ -251,11 +255,17 @@ class FP8AdamW:
                 "amax_m": self.amax_m.clone(), "amax_v": self.amax_v.clone(),
                 "m_fmt": self.m_fmt, "v_fmt": self.v_fmt,
                 "amax_history_m": None if self.hist_m is None else self.hist_m.clone(),
-                "amax_history_v": None if self.hist_v is None else self.hist_v.clone()}
+                "amax_history_v": None if self.hist_v is None else self.hist_v.clone(),
+                "sr_config": dict(self.sr_config)}
 
     def load_state_dict(self, sd: dict) -> None:
         if sd["m_fmt"] != self.m_fmt or sd["v_fmt"] != self.v_fmt:
             raise ValueError("moment formats differ")
+        if "sr_config" in sd and sd["sr_config"] != self.sr_config:
+            # the draws of step t depend on the seed, the draw width and the
+            # tensor ids: a different stream would not continue the run
+            raise ValueError("stochastic-rounding configuration differs: %r vs %r" % (sd["sr_config"],
+                                                                                       self.sr_config))
         with torch.no_grad():
             for dst, src in zip(self.params, sd["params"]):
                 dst.copy_(src)

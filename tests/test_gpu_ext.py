@@ -457,3 +457,30 @@ def test_sr_tensor_ids_key_the_draws(draws):
         r.compare()
     torch.cuda.synchronize()
     assert not torch.equal(r.M.m, plain.M.m)
+
+
+@DRAWS
+def test_checkpoint_resume_with_stochastic_rounding_is_bitwise(draws):
+    """Ten SR steps in one go equal five, a checkpoint, a fresh optimizer on
+    fresh buffers restored from it, and five more, bit for bit: the step
+    index, seed, draw width and tensor ids carry the random stream.  A
+    checkpoint refuses to load into an optimizer with another seed."""
+    kw = dict(stochastic_rounding=True, seed=777, sr_draw_bits=draws, subset=[])
+    a = ExtRun(60, **kw)
+    for _ in range(10):
+        a.step()
+    b = ExtRun(60, **kw)
+    for _ in range(5):
+        b.step()
+    sd = b.opt.state_dict()
+    c = ExtRun(60, **kw)
+    c.opt.load_state_dict(sd)
+    c.t = b.t
+    for _ in range(5):
+        c.step()
+    torch.cuda.synchronize()
+    for x in ("p", "m", "v", "scale_m", "scale_v", "amax_m", "amax_v"):
+        assert torch.equal(getattr(a.M, x).view(torch.uint8), getattr(c.M, x).view(torch.uint8)), x
+    other = ExtRun(60, stochastic_rounding=True, seed=778, sr_draw_bits=draws, subset=[])
+    with pytest.raises(ValueError):
+        other.opt.load_state_dict(sd)
