@@ -186,7 +186,7 @@ const char* fp8adam_strerror(int code);
  * conversion (cvt.rs, four codes per instruction, one Philox4x32-10 call per
  * eight elements).  Code of element j: up iff floor((|x|-lo)/(hi-lo) * 2^16)
  * + r >= 2^16, r the draw of code j % 4 of word 2*((j/4) % 2) + (0 for m, 1
- * for v) of the call with counter (j/8 low, j/8 high, tensor, step), draws as
+ * for v) of the call with counter (j/8 low, j/8 high, id(i), step), draws as
  * fp8adam_encode_sr16 takes them.  The probability of rounding up is the
  * exact one rounded down to a multiple of 2^-16. */
 #define FP8ADAM_FLAG_SR_DRAW16 32u
