@@ -222,9 +222,13 @@ def test_prepass_only_equals_default_kernel():
         assert torch.equal(getattr(a.M, x).view(torch.uint8), getattr(b.M, x).view(torch.uint8)), x
 
 
-def test_options_with_fp32_moments_and_current_scaling():
+@DRAWS
+def test_options_with_fp32_moments_and_current_scaling(draws):
+    """One fp32 moment (per-thread kernel) and current scaling (an amax
+    pre-pass every step), with a margin, stochastic rounding, a loss scale and
+    clipping."""
     r = ExtRun(47, mf=oracle.FP32, vf=oracle.E5M2, margin_v=1, stochastic_rounding=True, seed=5,
-               jit_every_step=True)
+               jit_every_step=True, sr_draw_bits=draws)
     r.flags |= oracle.FLAG_JIT_EVERY_STEP
     for _ in range(4):
         r.step(loss_scale=4.0, max_norm=0.5)
@@ -484,3 +488,17 @@ def test_checkpoint_resume_with_stochastic_rounding_is_bitwise(draws):
     other = ExtRun(60, stochastic_rounding=True, seed=778, sr_draw_bits=draws, subset=[])
     with pytest.raises(ValueError):
         other.opt.load_state_dict(sd)
+
+
+@pytest.mark.parametrize("fmts", [(oracle.E4M3, oracle.E4M3), (oracle.E5M2, oracle.E5M2)], ids=["m4v4", "m5v5"])
+@pytest.mark.parametrize("tma", [True, False], ids=["staged", "vector"])
+def test_sr16_same_format_pairs_with_current_scaling(fmts, tma):
+    """16-bit-draw stochastic rounding for the pairs with one format for both
+    moments (the staged kernel's E4M3/E4M3 and E5M2/E5M2 instances, or the
+    per-thread kernel), with current scaling: bit for bit over four steps."""
+    r = ExtRun(61, mf=fmts[0], vf=fmts[1], stochastic_rounding=True, seed=99, sr_draw_bits=16, tma=tma,
+               jit_every_step=True)
+    r.flags |= oracle.FLAG_JIT_EVERY_STEP
+    for _ in range(4):
+        r.step()
+        r.compare()
