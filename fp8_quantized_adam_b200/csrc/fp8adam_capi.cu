@@ -220,6 +220,25 @@ ExtFn pick_amax_ext(int mf, int vf) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+// A staged step kernel launched with programmatic dependent launch: it may
+// start while the previous kernel on the stream finishes (it waits for that
+// kernel's writes with griddepcontrol.wait).
+template <typename Args>
+cudaError_t launch_staged_pdl(void (*fn)(const Args, uint32_t*), dim3 grid, dim3 block, cudaStream_t st,
+                              const Args& args, uint32_t* err) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = kTmaSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, args, err);
+}
+
 static_assert(FP8ADAM_FLAG_UPDATE_FROM_STORED == kExtFromStored && FP8ADAM_FLAG_STOCHASTIC_ROUNDING == kExtStochastic &&
                   FP8ADAM_FLAG_SR_DRAW16 == kExtSrDraw16,
               "the step passes these flag bits to the kernels unchanged");
@@ -658,8 +677,9 @@ static float host_multiplier(const fp8adam_step_params& p) {
 // `cur` (a scheduled step): the kernels take the constants and per-step
 // options from that device entry instead of `p`; whether the pre-passes run
 // is then decided per schedule (grad norm) or per context (JIT amax).
-// `pdl`: launch the staged default step with programmatic dependent launch
-// (the steps of fp8adam_step / fp8adam_step_ex, back to back on a stream).
+// `pdl`: launch the staged step kernel (default or options) with
+// programmatic dependent launch (the steps of fp8adam_step /
+// fp8adam_step_ex, back to back on a stream).
 static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaStream_t st, int32_t c0, int32_t c1,
                           bool first, const SchedEntry* cur = nullptr, bool pdl = false) {
   if (c1 <= c0) return FP8ADAM_OK;  // only empty tensors
@@ -708,20 +728,8 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
       a.amax_in_v = reinterpret_cast<const uint32_t*>(ctx->amax_v);
     }
     if (ctx->tma && pdl) {
-      // the kernel may start while the previous kernel on the stream finishes
-      // (it waits for that kernel's writes with griddepcontrol.wait)
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[0].val.programmaticStreamSerializationAllowed = 1;
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = grid;
-      cfg.blockDim = block;
-      cfg.dynamicSmemBytes = kTmaSmemBytes;
-      cfg.stream = st;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      uint32_t* err = ctx->d_error;
-      if (cudaLaunchKernelEx(&cfg, pick_tma(ctx->m_fmt, ctx->v_fmt, stats), a, err) != cudaSuccess) {
+      if (launch_staged_pdl(pick_tma(ctx->m_fmt, ctx->v_fmt, stats), grid, block, st, a, ctx->d_error) !=
+          cudaSuccess) {
         cudaGetLastError();
         return FP8ADAM_ERR_CUDA;
       }
@@ -782,12 +790,20 @@ static int run_step_range(fp8adam_ctx* ctx, const fp8adam_step_params& p, cudaSt
   }
   e.s = a;
   const int srk = sr_kind_of(e.flags);
-  if (ctx->tma && srk && !(e.flags & FP8ADAM_FLAG_UPDATE_FROM_STORED) && !ctx->d_bf16 && e.grad_mult == nullptr &&
-      e.gm_const == 1.0f)
-    pick_ext_tma_sr_lean(ctx->m_fmt, ctx->v_fmt, stats, srk)<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
-  else if (ctx->tma)
-    pick_ext_tma(ctx->m_fmt, ctx->v_fmt, stats, srk)<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
-  else
+  if (ctx->tma) {
+    const bool lean = srk && !(e.flags & FP8ADAM_FLAG_UPDATE_FROM_STORED) && !ctx->d_bf16 && e.grad_mult == nullptr &&
+                      e.gm_const == 1.0f;
+    const ExtTmaFn fn = lean ? pick_ext_tma_sr_lean(ctx->m_fmt, ctx->v_fmt, stats, srk)
+                             : pick_ext_tma(ctx->m_fmt, ctx->v_fmt, stats, srk);
+    if (pdl) {
+      if (launch_staged_pdl(fn, grid, block, st, e, ctx->d_error) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8ADAM_ERR_CUDA;
+      }
+    } else {
+      fn<<<grid, block, kTmaSmemBytes, st>>>(e, ctx->d_error);
+    }
+  } else
     pick_ext(ctx->m_fmt, ctx->v_fmt, stats)<<<grid, block, 0, st>>>(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return last_error();

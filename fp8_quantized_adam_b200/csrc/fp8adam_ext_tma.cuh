@@ -144,13 +144,23 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   __shared__ uint32_t red[4][kThreads / 32];
   __shared__ int abort_flag;
 
-  if (*(volatile const uint32_t*)err) return;  // an earlier CTA timed out: stop at once
-  if (a.skip && *a.skip) return;              // a non-finite gradient: the step is skipped
-  if (a.s.cur && !a.s.cur->valid) return;     // the schedule ran out
+  // The chunk and tensor tables are static (written at create), so they are
+  // read before the previous kernel in the stream has finished.  With
+  // programmatic dependent launch this grid starts while that kernel's last
+  // CTAs still run: every CTA lets the next grid start once all of this
+  // grid's CTAs have started, then waits for the previous grid's writes
+  // before it reads anything a step writes (the error word, the skip flag,
+  // the schedule entry, the multiplier, scales, amax, params, moments).
+  // Launched without it, both instructions return at once.
   const Chunk ch = a.s.chunks[blockIdx.x];
   const int ti = ch.tensor;
   FP8ADAM_BOUNDS(ti >= 0 && ti < a.s.num_tensors);
   const TensorDesc td = a.s.tensors[ti];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (*(volatile const uint32_t*)err) return;  // an earlier CTA timed out: stop at once
+  if (a.skip && *a.skip) return;              // a non-finite gradient: the step is skipped
+  if (a.s.cur && !a.s.cur->valid) return;     // the schedule ran out
   const int64_t e0 = ch.start, e1 = ch.start + ch.len;
   FP8ADAM_BOUNDS(e0 >= 0 && e0 <= e1 && e1 <= td.numel);
   // whole sub-tiles are staged when the tensor and its bf16 output (if any)
