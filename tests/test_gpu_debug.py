@@ -25,7 +25,10 @@ SEED = 51
 
 
 class Model:
-    def __init__(self, L):
+    """The C ABI on a seeded model; `opts` (fp8adam_options fields) creates
+    the context with fp8adam_create_ex."""
+
+    def __init__(self, L, opts=None):
         self.L = L
         self.specs = workloads.custom_layout(SIZES)
         self.M = workloads.FlatModel(self.specs, torch.device("cuda:0"))
@@ -37,8 +40,23 @@ class Model:
             arr[i] = capi.fp8adam_tensor(M.view(M.p, i).data_ptr(), M.view(M.g, i).data_ptr(),
                                          M.view(M.m, i).data_ptr(), M.view(M.v, i).data_ptr(), self.specs[i].numel)
         out = ctypes.c_void_p()
-        assert L.fp8adam_create(arr, M.T, M.scale_m.data_ptr(), M.scale_v.data_ptr(), M.amax_m.data_ptr(),
-                                M.amax_v.data_ptr(), 0, 1, 0, ctypes.byref(out)) == capi.OK
+        if opts is None:
+            assert L.fp8adam_create(arr, M.T, M.scale_m.data_ptr(), M.scale_v.data_ptr(), M.amax_m.data_ptr(),
+                                    M.amax_v.data_ptr(), 0, 1, 0, ctypes.byref(out)) == capi.OK
+        else:
+            kw = dict(opts)
+            self.keep = []  # host arrays and device buffers the options point to
+            if kw.get("amax_history_len", 0) > 1:
+                h = torch.zeros(2, kw["amax_history_len"], M.T, device="cuda:0")
+                self.keep.append(h)
+                kw["amax_history_m"], kw["amax_history_v"] = h[0].data_ptr(), h[1].data_ptr()
+            if "sr_counter_ids" in kw:
+                ids = (ctypes.c_uint32 * M.T)(*kw["sr_counter_ids"])
+                self.keep.append(ids)
+                kw["sr_counter_ids"] = ctypes.cast(ids, ctypes.c_void_p)
+            o = capi.fp8adam_options(scale_m=M.scale_m.data_ptr(), scale_v=M.scale_v.data_ptr(),
+                                     amax_m=M.amax_m.data_ptr(), amax_v=M.amax_v.data_ptr(), m_fmt=0, v_fmt=1, **kw)
+            assert L.fp8adam_create_ex(arr, M.T, ctypes.byref(o), ctypes.byref(out)) == capi.OK
         self.ctx = out
         self.stream = torch.cuda.current_stream().cuda_stream
 
@@ -72,8 +90,8 @@ def _same(a, b):
     return all(torch.equal(x.view(torch.uint8), y.view(torch.uint8)) for x, y in zip(a, b))
 
 
-def _release_state(steps):
-    r = Model(capi.lib())
+def _release_state(steps, opts=None):
+    r = Model(capi.lib(), opts)
     for t in range(1, steps + 1):
         assert r.step(t) == capi.OK
     assert r.check() == capi.OK
@@ -85,6 +103,23 @@ def _release_state(steps):
 def test_debug_build_matches_release_and_reports_nothing():
     want = _release_state(4)
     d = Model(capi.debug_lib())
+    for t in range(1, 5):
+        assert d.step(t) == capi.OK
+    assert d.check() == capi.OK
+    assert _same(d.state(), want)
+    d.close()
+
+
+@pytest.mark.parametrize("opts", [
+    dict(flags=capi.FLAG_STOCHASTIC_ROUNDING | capi.FLAG_SR_DRAW16, seed=9, sr_counter_ids=[5, 1, 9, 2, 7, 3]),
+    dict(flags=capi.FLAG_STOCHASTIC_ROUNDING, seed=9, amax_history_len=3, margin_m=1, margin_v=2)],
+    ids=["sr16_ids", "sr32_history_margin"])
+def test_debug_build_matches_release_with_options(opts):
+    """The option kernels (stochastic rounding with 16-bit draws and counter
+    ids; with 32-bit draws, an amax history and margins) in the debug build:
+    the release build's results bit for bit, and no bounds violation."""
+    want = _release_state(4, opts)
+    d = Model(capi.debug_lib(), opts)
     for t in range(1, 5):
         assert d.step(t) == capi.OK
     assert d.check() == capi.OK
