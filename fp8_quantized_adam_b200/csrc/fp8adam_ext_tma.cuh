@@ -179,18 +179,20 @@ fp8adam_step_ext_tma_kernel(const ExtArgs a, uint32_t* err) {
   if constexpr (SRK == 1) su = sr_chunk(a, sg.sr_id, sg.t_lo, e0 >> 1);
   if constexpr (SRK == 2) su = sr_chunk(a, sg.sr_id, sg.t_lo, e0 >> 3);
   uint32_t w1m = 0, w1v = 0;  // 16-bit draws: the words of this thread's second group of the stage
-  if (!tma_run(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
+  if (!tma_run(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i, int h) {
         uint32_t wm = 0, wv = 0;
         if constexpr (SRK == 2) {
-          if (j < 4 * kThreads) {
+          if (h == 0) {
             // The stage's first group of thread t is elements i .. i+3 (i = 8q
             // for even t, 8q + 4 for odd t), its second i + 1024 .. i + 1027.
             // One Philox call per thread and stage: even t takes the call of
             // its first group's eight elements (its own four and those of
             // t + 1), odd t that of its second group's (those of t - 1 and its
             // own); each passes the neighbour the two words it needs.
+            // the counter's low word: i/8, or (i + 1024)/8 = i/8 + 128 for odd
+            // t (i = 8q + 4); modulo 2^32 like the counter word itself
             const bool odd = (threadIdx.x & 1u) != 0;
-            const uint4 w = sr_words_chunk(a, su, (uint32_t)((odd ? i + 4 * kThreads : i) >> 3));
+            const uint4 w = sr_words_chunk(a, su, (uint32_t)(i >> 3) + (odd ? (uint32_t)(4 * kThreads / 8) : 0u));
             const uint32_t g0 = __shfl_xor_sync(0xFFFFFFFFu, odd ? w.x : w.z, 1);
             const uint32_t g1 = __shfl_xor_sync(0xFFFFFFFFu, odd ? w.y : w.w, 1);
             wm = odd ? g0 : w.x;

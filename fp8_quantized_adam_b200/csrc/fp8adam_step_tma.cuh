@@ -157,9 +157,10 @@ __device__ __forceinline__ void tma_issue(const TensorDesc& td, int64_t e0, int 
 // set-up while the first copies are in flight:
 // - tma_begin initialises the stage barriers and has thread 0 issue the
 //   first kStages sub-tiles;
-// - tma_run then has every thread call body(st, j, i) for its 2 groups of 4
-//   elements of each sub-tile (stage st, stage offset j, global element i),
-//   refilling each stage once all threads are done with it.
+// - tma_run then has every thread call body(st, j, i, h) for its 2 groups of
+//   4 elements of each sub-tile (stage st, stage offset j, global element i,
+//   group h = 0 or 1, a constant once the loop is unrolled), refilling each
+//   stage once all threads are done with it.
 // `full` and `abort_flag` live in the kernel's shared memory.  tma_run
 // returns false if a wait gave up: then bit 0 of *err is set and the copies
 // still in flight have been waited for (bounded), so the CTA can return.
@@ -193,7 +194,7 @@ __device__ __forceinline__ bool tma_run(const TensorDesc& td, int64_t e0, int ns
 #pragma unroll
     for (int h = 0; h < kSub / (4 * kThreads); ++h) {  // 2 groups of 4 elements per thread
       const int j = h * (4 * kThreads) + 4 * (int)threadIdx.x;
-      body(stage[s], j, e0 + (int64_t)k * kSub + j);
+      body(stage[s], j, e0 + (int64_t)k * kSub + j, h);
     }
     __syncthreads();  // every thread is done reading stage s
     if (threadIdx.x == 0 && k + kStages < nsub) {
@@ -258,7 +259,7 @@ fp8adam_step_tma_kernel(const StepArgs a, uint32_t* err) {
   float am = 0.0f, av = 0.0f;
   uint32_t flushed = 0, sat = 0;
 
-  if (!tma_run(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i) {
+  if (!tma_run(td, e0, nsub, stage, full, abort_flag, err, [&](const TmaStage& st, int j, int64_t i, int) {
         consume4<MF, VF, STATS>(st, j, td, i, c, inv_s_m, inv_s_v, s_m_new, s_v_new, am, av, flushed, sat);
       }))
     return;
