@@ -42,14 +42,14 @@ FALLBACK_HBM_GBS = 6650.0
 # step kernel in steady state: two consecutive launches on the pair_2x256m
 # layout (536,870,912 params, 7.5 GB of traffic, far larger than L2) captured
 # with --cache-control none, so the dirty L2 lines a launch leaves are written
-# back inside the next one: 8.0009 B read + 5.9946 B written per param.  With
-# the cache flushed before each launch instead, the writes come to 5.886 B per
+# back inside the next one: 8.0015 B read + 5.9949 B written per param.  With
+# the cache flushed before each launch instead, the writes come to 5.887 B per
 # param: L2_RESIDUE bytes of a launch's writes are still dirty in L2 at its
 # exit.  Both are per launch and valid while the kernel's device code hashes
 # to KERNEL_SHA (null otherwise).
-TRAFFIC_PER_PARAM = 13.99548
-L2_RESIDUE = 61.2e6
-KERNEL_SHA = "cb7246f1694ca91f"
+TRAFFIC_PER_PARAM = 13.99641
+L2_RESIDUE = 60.7e6
+KERNEL_SHA = "f49bdeb639a8eda0"
 
 
 def _code_only(src: str) -> str:
