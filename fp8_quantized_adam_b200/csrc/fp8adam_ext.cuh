@@ -285,6 +285,7 @@ __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& 
   tv.load(td.v, i);
   const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
   uint32_t pbw[8];
+  uint4 w16 = make_uint4(0, 0, 0, 0);  // 16-bit draws: the words of the current eight elements
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     float mo[4], vo[4], mn[4], vn[4], mu[4], vu[4];
@@ -300,10 +301,13 @@ __device__ __forceinline__ void ext_group16(const ExtArgs& a, const TensorDesc& 
       rmj[0] = r0.x; rmj[1] = r0.z; rmj[2] = r1.x; rmj[3] = r1.z;
       rvj[0] = r0.y; rvj[1] = r0.w; rvj[2] = r1.y; rvj[3] = r1.w;
     } else if (srk == 2) {  // i + 4k is a multiple of 4: one word for the four m codes, one for the v codes
-      const uint4 r = sr_words(a, sg.sr_id, sg.t_lo, (i + 4 * k) >> 3);
-      const bool second = (((i + 4 * k) >> 2) & 1) != 0;
-      rmj[0] = rmj[1] = rmj[2] = rmj[3] = second ? r.z : r.x;
-      rvj[0] = rvj[1] = rvj[2] = rvj[3] = second ? r.w : r.y;
+      // one call per eight elements: a new one unless this group is the
+      // second half of the previous group's eight
+      const int64_t e = i + 4 * k;
+      if (k % 2 == 0 || (e & 7) == 0) w16 = sr_words(a, sg.sr_id, sg.t_lo, e >> 3);
+      const bool second = ((e >> 2) & 1) != 0;
+      rmj[0] = rmj[1] = rmj[2] = rmj[3] = second ? w16.z : w16.x;
+      rvj[0] = rvj[1] = rvj[2] = rvj[3] = second ? w16.w : w16.y;
     }
     uint32_t qm[4], qv[4];
 #pragma unroll
