@@ -184,11 +184,13 @@ const char* fp8adam_strerror(int code);
 /* With FP8ADAM_FLAG_STOCHASTIC_ROUNDING (INVALID_ARG without it): 16-bit
  * draws instead of 32-bit ones, rounded by the B200's stochastic-rounding
  * conversion (cvt.rs, four codes per instruction, one Philox4x32-10 call per
- * eight elements).  Code of element j: up iff floor((|x|-lo)/(hi-lo) * 2^16)
- * + r >= 2^16, r the draw of code j % 4 of word 2*((j/4) % 2) + (0 for m, 1
- * for v) of the call with counter (j/8 low, j/8 high, id(i), step), draws as
- * fp8adam_encode_sr16 takes them.  The probability of rounding up is the
- * exact one rounded down to a multiple of 2^-16. */
+ * eight elements).  The code of element j of tensor i rounds up iff
+ * floor((|x|-lo)/(hi-lo) * 2^16) + r >= 2^16, with r the draw of code j % 4
+ * of word 2*((j/4) % 2) + (0 for m, 1 for v) of the Philox4x32-10 call with
+ * counter (j/8 low, j/8 high, id(i), step low 32 bits) and key (seed low,
+ * seed high), draws as fp8adam_encode_sr16 takes them; id(i) and the seed
+ * are fp8adam_options' (sr_counter_ids, seed).  The probability of rounding
+ * up is the exact one rounded down to a multiple of 2^-16. */
 #define FP8ADAM_FLAG_SR_DRAW16 32u
 
 typedef struct {
